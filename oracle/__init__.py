@@ -1,0 +1,220 @@
+"""CPU oracle of the MoE layer hot path (test infrastructure only).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never loads it and
+shares no code with it: the arithmetic lives in ``moe_oracle.c`` (plain C,
+loops that follow the definitions, double accumulation), and this module only
+compiles that file with gcc and marshals numpy arrays through ctypes.
+
+bf16 tensors travel as ``np.uint16`` arrays holding the bf16 bit patterns;
+fp32 tensors as ``np.float32``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32 = 0
+BF16 = 1
+
+_lib = None
+# The mutation tests point a fresh process at a deliberately broken build.
+_lib_path = os.environ.get("MOE_ORACLE_LIB") or _LIB
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into liboracle.so (no fused multiply-add, no fast math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+             "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def use_library(path: str | None) -> None:
+    """Point the wrappers at another build of the oracle (None: the default one).
+
+    The mutation tests compile deliberately broken copies of moe_oracle.c and
+    check that the pins reject them."""
+    global _lib, _lib_path
+    _lib, _lib_path = None, (path or _LIB)
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if _lib_path == _LIB:
+            build()
+        lib = ctypes.CDLL(_lib_path)
+        p, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        lib.oracle_gate.argtypes = [p, p, i32, i32, i32, i32, p]
+        lib.oracle_gate.restype = None
+        lib.oracle_route.argtypes = [p, p, i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p]
+        lib.oracle_route.restype = i32
+        lib.oracle_dispatch.argtypes = [p, i32, i32, i32, i32, p, i32, p]
+        lib.oracle_dispatch.restype = None
+        lib.oracle_expert_ffn_row.argtypes = [p, p, p, i32, i32, i32, i32, p, p]
+        lib.oracle_expert_ffn_row.restype = None
+        lib.oracle_expert_ffn.argtypes = [p, p, p, i32, i32, i32, i32, p, p, p]
+        lib.oracle_expert_ffn.restype = None
+        lib.oracle_combine.argtypes = [p, i32, i32, i32, i32, p, p, p]
+        lib.oracle_combine.restype = None
+        lib.oracle_popularity_update.argtypes = [p, i32, p, i32, i64, p, i32, p]
+        lib.oracle_popularity_update.restype = i32
+        lib.oracle_round_bf16.argtypes = [ctypes.c_double]
+        lib.oracle_round_bf16.restype = ctypes.c_uint16
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.uint16:
+        return BF16
+    if a.dtype == np.float32:
+        return F32
+    raise TypeError(f"oracle tensors are float32 or bf16 bits (uint16), got {a.dtype}")
+
+
+def _c(a, dtype=None):
+    a = np.ascontiguousarray(a if dtype is None else a.astype(dtype, copy=False))
+    return a
+
+
+def round_bf16(v: float) -> int:
+    """bf16 bits of the double ``v`` rounded once, to nearest even."""
+    return int(_load().oracle_round_bf16(float(v)))
+
+
+def gate(x: np.ndarray, Wg: np.ndarray) -> np.ndarray:
+    """logits[T,E] = x[T,d] . Wg[E,d]^T, double accumulation, fp32 result."""
+    x, Wg = _c(x), _c(Wg)
+    dt = _dtype_code(x)
+    assert _dtype_code(Wg) == dt and x.shape[1] == Wg.shape[1]
+    T, d = x.shape
+    E = Wg.shape[0]
+    out = np.empty((T, E), np.float32)
+    _load().oracle_gate(_ptr(x), _ptr(Wg), dt, T, d, E, _ptr(out))
+    return out
+
+
+def route(logits: np.ndarray, bias, k: int, capacity: int = 0, rank_major: bool = False):
+    """Top-k routing with capacity; returns a dict of the route outputs.
+
+    ``row_slot`` is returned trimmed to R = offsets[E] rows.
+    """
+    logits = _c(logits, np.float32)
+    T, E = logits.shape
+    b = None if bias is None else _c(bias, np.float32)
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float32)
+    counts = np.empty(E, np.int32)
+    kept = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    slot_row = np.empty((T, k), np.int32)
+    row_slot = np.full(max(T * k, 1), -1, np.int32)
+    nd = np.zeros(1, np.int32)
+    rc = _load().oracle_route(_ptr(logits), _ptr(b), T, E, k, int(capacity), int(rank_major),
+                              _ptr(ids), _ptr(w), _ptr(counts), _ptr(kept), _ptr(offsets),
+                              _ptr(slot_row), _ptr(row_slot), _ptr(nd))
+    if rc != 0:
+        raise ValueError("oracle_route: invalid sizes")
+    R = int(offsets[E])
+    return dict(ids=ids, w=w, counts=counts, kept=kept, offsets=offsets, slot_row=slot_row,
+                row_slot=row_slot[:R].copy(), n_dropped=int(nd[0]))
+
+
+def dispatch(x: np.ndarray, k: int, row_slot: np.ndarray) -> np.ndarray:
+    """Xp[row] = x[row_slot[row] // k]."""
+    x = _c(x)
+    dt = _dtype_code(x)
+    T, d = x.shape
+    rs = _c(row_slot, np.int32)
+    R = rs.shape[0]
+    Xp = np.empty((R, d), x.dtype)
+    _load().oracle_dispatch(_ptr(x), dt, T, d, k, _ptr(rs), R, _ptr(Xp))
+    return Xp
+
+
+def expert_ffn(Xp: np.ndarray, W1: np.ndarray, W2: np.ndarray, offsets: np.ndarray,
+               want_h: bool = False):
+    """Yp (and optionally H) for every grouped row; W1 [E,F,d], W2 [E,d,F]."""
+    Xp, W1, W2 = _c(Xp), _c(W1), _c(W2)
+    dt = _dtype_code(Xp)
+    E, F, d = W1.shape
+    assert W2.shape == (E, d, F) and Xp.shape[1] == d
+    off = _c(offsets, np.int32)
+    R = int(off[E])
+    Yp = np.zeros((Xp.shape[0], d), Xp.dtype)
+    H = np.zeros((Xp.shape[0], F), Xp.dtype) if want_h else None
+    _load().oracle_expert_ffn(_ptr(Xp), _ptr(W1), _ptr(W2), dt, E, d, F, _ptr(off), _ptr(H),
+                              _ptr(Yp))
+    Yp = Yp[:R]
+    return (Yp, H[:R]) if want_h else Yp
+
+
+def expert_ffn_rows(rows: np.ndarray, experts, W1: np.ndarray, W2: np.ndarray,
+                    want_h: bool = False):
+    """FFN of selected rows: rows[n,d] each through experts[n]."""
+    rows, W1, W2 = _c(rows), _c(W1), _c(W2)
+    dt = _dtype_code(rows)
+    E, F, d = W1.shape
+    n = rows.shape[0]
+    Y = np.empty((n, d), rows.dtype)
+    H = np.empty((n, F), rows.dtype) if want_h else None
+    lib = _load()
+    es = rows.itemsize
+    for i, e in enumerate(np.asarray(experts).tolist()):
+        hp = None if H is None else ctypes.c_void_p(H.ctypes.data + i * F * es)
+        lib.oracle_expert_ffn_row(ctypes.c_void_p(rows.ctypes.data + i * d * es), _ptr(W1),
+                                  _ptr(W2), dt, int(e), d, F, hp,
+                                  ctypes.c_void_p(Y.ctypes.data + i * d * es))
+    return (Y, H) if want_h else Y
+
+
+def combine(Yp: np.ndarray, T: int, k: int, slot_row: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """y[t] = sum_j w[t,j] Yp[slot_row[t,j]] over kept slots."""
+    Yp = _c(Yp)
+    dt = _dtype_code(Yp)
+    d = Yp.shape[1]
+    sr, ww = _c(slot_row, np.int32), _c(w, np.float32)
+    y = np.empty((T, d), Yp.dtype)
+    _load().oracle_combine(_ptr(Yp), dt, T, d, k, _ptr(sr), _ptr(ww), _ptr(y))
+    return y
+
+
+def popularity_update(counts: np.ndarray, hist: np.ndarray, step: int, P: int):
+    """Updates ``hist`` [W,E] in place; returns (mean[E] fp32, hot[P] int32)."""
+    counts = _c(counts, np.int32)
+    assert hist.dtype == np.int32 and hist.flags.c_contiguous
+    W, E = hist.shape
+    mean = np.empty(E, np.float32)
+    hot = np.empty(max(P, 1), np.int32)
+    rc = _load().oracle_popularity_update(_ptr(counts), E, _ptr(hist), W, int(step), _ptr(mean),
+                                          P, _ptr(hot))
+    if rc != 0:
+        raise ValueError("oracle_popularity_update: invalid sizes")
+    return mean, hot[:P].copy()
+
+
+def layer(x, Wg, W1, W2, bias, k, capacity=0, logits=None):
+    """Whole layer: gate (unless logits are given), route, dispatch, FFN, combine."""
+    if logits is None:
+        logits = gate(x, Wg)
+    r = route(logits, bias, k, capacity)
+    Xp = dispatch(x, k, r["row_slot"])
+    Yp = expert_ffn(Xp, W1, W2, r["offsets"])
+    y = combine(Yp, x.shape[0], k, r["slot_row"], r["w"])
+    return dict(logits=logits, Xp=Xp, Yp=Yp, y=y, **r)

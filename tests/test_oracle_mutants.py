@@ -1,0 +1,59 @@
+"""The oracle's pins must reject plausible mistakes (CPU only).
+
+Each case plants one mistake in a copy of oracle/moe_oracle.c, builds it, and
+runs the pin suite against that build in a fresh process: the suite has to fail.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+from conftest import ROOT
+
+SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
+
+MUTANTS = {
+    "tie_to_higher_index": ("if (best < 0 || z[e] > z[best]) best = e;",
+                            "if (best < 0 || z[e] >= z[best]) best = e;"),
+    "weights_not_shifted": ("(float)(exp((double)z[ids[(int64_t)t * k + j]] - zmax) / denom)",
+                            "(float)(exp((double)z[ids[(int64_t)t * k + j]]) / denom)"),
+    "capacity_off_by_one": ("if (capacity <= 0 || p < capacity) {",
+                            "if (capacity <= 0 || p <= capacity) {"),
+    "inclusive_offsets": ("        offsets[e] = total;\n        total += kept[e];",
+                          "        total += kept[e];\n        offsets[e] = total;"),
+    "bias_ignored": ("float b = bias ? bias[e] : 0.0f;", "float b = 0.0f;"),
+    "w1_transposed": ("load_elem(W1, dtype, w1base + (int64_t)f * d + c)",
+                      "load_elem(W1, dtype, w1base + (int64_t)c * F + f)"),
+    "relu_missing": ("double r = acc > 0.0 ? acc : 0.0;", "double r = acc;"),
+    "h_not_rounded": ("h[f] = bf16_bits_to_double(double_to_bf16_bits(r));", "h[f] = r;"),
+    "h_fp32_not_rounded": ("h[f] = (double)(float)r;", "h[f] = r;"),
+    "w2_wrong_expert": ("w2base = (int64_t)e * d * F;", "w2base = 0;"),
+    "combine_first_weight_only": ("double wj = (double)w[(int64_t)t * k + j];",
+                                  "double wj = (double)w[(int64_t)t * k];"),
+    "dispatch_wrong_token": ("int t = row_slot[row] / k;", "int t = row_slot[row] % T;"),
+    "gate_transposed": ("load_elem(Wg, dtype, (int64_t)e * d + c)",
+                        "load_elem(Wg, dtype, (int64_t)c * E + e)"),
+    "window_not_clamped": ("int64_t n = step + 1 < W ? step + 1 : W;", "int64_t n = W;"),
+    "hot_tie_to_higher": ("if (best < 0 || sum[e] > sum[best]) best = e;",
+                          "if (best < 0 || sum[e] >= sum[best]) best = e;"),
+    "bf16_double_rounding": ("double a = fabs(v);", "double a = (double)(float)fabs(v);"),
+    "bf16_ties_away": ("double r = rint(ldexp(a, -q));", "double r = round(ldexp(a, -q));"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    mutated = tmp_path / "moe_oracle_mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib = tmp_path / "liboracle_mutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+                           "-fPIC", "-shared", "-o", str(lib), str(mutated), "-lm"])
+    env = dict(os.environ, MOE_ORACLE_LIB=str(lib))
+    res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                          os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert res.returncode != 0, f"pins accepted the mutant {name}:\n{res.stdout[-2000:]}"
