@@ -1,0 +1,424 @@
+"""Benchmark of the MoE layer hot path: tokens/s on B200, roofline fractions.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = gate projection, top-k routing with capacity, popularity window
+update, dispatch (input encode), expert FC-ReLU-FC and combine (output decode)
+over one batch of T tokens, every stage a kernel of libmoe.so behind the C ABI.
+Inputs are seeded synthetic tensors of the workload's shapes (workloads.py);
+weights are random-init and resident in HBM.  The timed region is bracketed by
+a barrier and a device synchronize on both sides and timed with CUDA events on
+the launching stream; with N ranks (torchrun, one GPU each, independent
+per-rank batches: weak scaling) the time is the max over ranks and the only
+collective in a step is the all_reduce of the per-expert counts that keeps the
+popularity statistic global.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from routing_dispatch_expert_fp32_b200 import workloads as wl  # noqa: E402
+
+DEFAULT_WORKLOAD = "skewed_drops"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=0, help="timed steps (0: workload default)")
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=0, help="override T (bw_sweep sizes)")
+    ap.add_argument("--no-bias", action="store_true", help="bw_sweep without the Zipf bias")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def workload_of(args) -> wl.Workload:
+    w = wl.WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.with_(T=args.tokens)
+    if args.no_bias:
+        w = w.with_(zipf_s=None)
+    return w
+
+
+def default_steps(w: wl.Workload) -> int:
+    # about 2-4 s of timed work on one B200
+    return {"tiny_fp32": 20000, "skewed_drops": 4000, "multistep_window": 400,
+            "fine_grained": 300, "bw_sweep": 1000}[w.name]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def config_of(w: wl.Workload, n: int):
+    c = {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "F": w.F,
+         "capacity": w.capacity, "zipf_s": w.zipf_s, "global_batch_tokens": w.T * n,
+         "parallelism": f"dp{n}" if n > 1 else "single",
+         "l2": "inputs larger than L2: expert weights read every step exceed 126 MB"
+               if not w.identity_experts else
+               "inputs larger than L2: x and the grouped rows exceed 126 MB"}
+    if w.identity_experts:
+        c["experts"] = "identity"
+    if w.steps > 1:
+        c["popularity_window"] = w.W
+    return c
+
+
+# --------------------------------------------------------------- clocks ---
+class ClockSampler:
+    """nvidia-smi samples during the timed region (reads only)."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc, self.lines = index, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ----------------------------------------------------------- reference ---
+def cpu_oracle_run(w: wl.Workload, target_s: float):
+    """The oracle as it stands on a bounded token sample of the workload:
+    gate, route (capacity rescaled to the sample), dispatch, FFN, combine."""
+    import oracle
+
+    weights = wl.make_weights(w)
+    inp = wl.make_step(w, 0)
+
+    def run(n):
+        x = inp["x"][:n]
+        cap = 0
+        if w.capacity_factor is not None:
+            cap = int(np.ceil(float(w.capacity_factor) * n * w.k / w.E))
+        t0 = time.perf_counter()
+        if w.identity_experts:
+            r = oracle.route(inp["logits"][:n], inp["bias"], w.k, cap)
+            Xp = oracle.dispatch(x, w.k, r["row_slot"])
+            oracle.combine(Xp, n, w.k, r["slot_row"], r["w"])
+        else:
+            oracle.layer(x, weights.get("Wg"), weights["W1"], weights["W2"], inp["bias"], w.k,
+                         cap)
+        return time.perf_counter() - t0
+
+    n = min(w.T, 8)
+    dt = run(n)
+    while dt < target_s / 8 and n < w.T:
+        n = min(w.T, n * 4)
+        dt = run(n)
+    if dt < target_s and n < w.T:
+        n = min(w.T, max(n + 1, int(n * target_s / max(dt, 1e-6))))
+        dt = run(n)
+    return n / dt, n, dt
+
+
+def reference_arm(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    steps = args.steps or 3
+    times = []
+    n = 0
+    rate = 0.0
+    per = args.cpu_seconds / max(1, steps)
+    for _ in range(args.warmup if args.warmup < 3 else 1):
+        pass
+    for _ in range(steps):
+        rate, n, dt = cpu_oracle_run(w, per)
+        times.append(dt)
+    value = n * len(times) / sum(times)
+    line = {"impl": "reference", "metric": "MoE layer tokens/s", "value": value,
+            "unit": "tokens/s", "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+            "data": "synthetic", "config": config_of(w, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"first {n} tokens of the batch per step, whole layer"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ ours ---
+def main():
+    args = parse()
+    w = workload_of(args)
+    if args.impl == "reference":
+        reference_arm(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from routing_dispatch_expert_fp32_b200 import moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    steps = args.steps or default_steps(w)
+    warmup = max(3, args.warmup)
+
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    to_dev = lambda a: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)  # noqa: E731
+                        if a.dtype == np.uint16 else torch.from_numpy(a)).cuda()
+    weights = {k: to_dev(v) for k, v in wl.make_weights(w, rank).items()}
+    nb = w.steps if w.steps > 1 else 2
+    batches = []
+    for s in range(nb):
+        inp = wl.make_step(w, s, rank)
+        batches.append({k: (None if v is None else to_dev(v)) for k, v in inp.items()})
+    layer = moe.MoELayer(w.T, w.d, w.E, w.k, w.F, tdt, capacity=w.capacity, W=w.W, P=w.P,
+                         identity_experts=w.identity_experts)
+    stream = torch.cuda.current_stream()
+    hook = None
+    if world > 1:
+        hook = lambda c: dist.all_reduce(c)  # noqa: E731  global popularity (sum over ranks)
+
+    def step(i, ev=None):
+        b = batches[i % nb]
+        if ev is None:
+            layer.forward(b["x"], weights.get("Wg"), weights.get("W1"), weights.get("W2"),
+                          b["bias"], logits=b.get("logits"), counts_hook=hook)
+            return
+        # same calls as MoELayer.forward, with an event after each stage
+        ev[0].record(stream)
+        logits = b.get("logits")
+        if logits is None:
+            moe.moe_gate(b["x"], weights["Wg"], layer.logits)
+            logits = layer.logits
+        ev[1].record(stream)
+        moe.moe_route(logits, b["bias"], w.k, w.capacity, layer.ids, layer.w, layer.counts,
+                      layer.kept, layer.offsets, layer.slot_row, layer.row_slot,
+                      layer.n_dropped, layer.workspace)
+        if hook is not None:
+            hook(layer.counts)
+        moe.moe_popularity_update(layer.counts, layer.hist, layer.step, layer.mean, layer.P,
+                                  layer.hot)
+        layer.step += 1
+        ev[2].record(stream)
+        moe.moe_dispatch(b["x"], w.k, layer.slot_row, layer.Xp)
+        ev[3].record(stream)
+        if not w.identity_experts:
+            moe.moe_expert_ffn(layer.Xp, weights["W1"], weights["W2"], layer.offsets, layer.H,
+                               layer.Yp)
+        ev[4].record(stream)
+        moe.moe_combine(layer.Yp, w.k, layer.slot_row, layer.w, layer.y)
+        ev[5].record(stream)
+
+    # R per batch (untimed): algorithmic work of each step
+    R_of = []
+    for i in range(nb):
+        step(i)
+        R_of.append(int(layer.offsets[-1].item()))
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- timed region (device time, events on the launching stream) ----
+    nev = 6
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(steps):
+        step(i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    stage_ms = np.zeros(nev - 1)
+    for e in evs:
+        stage_ms += np.array([e[j].elapsed_time(e[j + 1]) for j in range(nev - 1)])
+    stage_ms /= steps
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # ---- end to end: pinned host x -> device, layer, y -> pinned host ----
+    e2e_steps = max(10, steps // 4)
+    host_x = [batches[i]["x"].cpu().pin_memory() for i in range(nb)]
+    host_logits = [None if batches[i].get("logits") is None else
+                   batches[i]["logits"].cpu().pin_memory() for i in range(nb)]
+    host_y = torch.empty(w.T, w.d, dtype=tdt).pin_memory()
+    dx = torch.empty_like(batches[0]["x"])
+    dlog = None if host_logits[0] is None else torch.empty_like(batches[0]["logits"])
+    h2d = host_x[0].numel() * host_x[0].element_size() + (
+        0 if dlog is None else host_logits[0].numel() * 4)
+    d2h = host_y.numel() * host_y.element_size()
+
+    def e2e_step(i):
+        dx.copy_(host_x[i % nb], non_blocking=True)
+        if dlog is not None:
+            dlog.copy_(host_logits[i % nb], non_blocking=True)
+        b = batches[i % nb]
+        layer.forward(dx, weights.get("Wg"), weights.get("W1"), weights.get("W2"), b["bias"],
+                      logits=dlog, counts_hook=hook)
+        host_y.copy_(layer.y, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    dev_err = moe.moe_device_error()
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        R_mean = float(np.mean([R_of[i % nb] for i in range(steps)]))
+        names = ["gate", "route+popularity", "dispatch", "expert_ffn", "combine"]
+        es = 2 if w.dtype == "bf16" else 4
+        per = {}
+        alg = {
+            "gate": (2.0 * w.T * w.d * w.E, "flop") if not w.logits_direct else (0, "flop"),
+            "route+popularity": (w.T * w.E * 4 + w.T * w.k * 4 * 4 + R_mean * 4, "byte"),
+            "dispatch": (w.T * w.d * es + R_mean * w.d * es + w.T * w.k * 4, "byte"),
+            "expert_ffn": (4.0 * R_mean * w.d * w.F, "flop"),
+            "combine": (R_mean * w.d * es + w.T * w.d * es + w.T * w.k * 8, "byte"),
+        }
+        for j, n in enumerate(names):
+            amount, kind = alg[n]
+            ms = float(stage_ms[j])
+            ent = {"ms": ms}
+            if ms > 0 and amount:
+                if kind == "flop":
+                    ent["tflops"] = amount / (ms * 1e-3) / 1e12
+                    ent["frac_bf16_sustained"] = ent["tflops"] / peaks["bf16_tflops_sustained"]
+                else:
+                    ent["gbs"] = amount / (ms * 1e-3) / 1e9
+                    ent["frac_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
+            per[n] = ent
+        if w.identity_experts:
+            dom = "dispatch" if per["dispatch"]["ms"] >= per["combine"]["ms"] else "combine"
+            amount = alg[dom][0]
+            roof = {"bound": "hbm", "kernel": f"{dom}_kernel",
+                    "achieved": amount / (per[dom]["ms"] * 1e-3) / 1e9,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        else:
+            # the grouped GEMM: two launches per step, 2*R*d*F flops each
+            launch_ms = per["expert_ffn"]["ms"] / 2
+            roof = {"bound": "tensor", "kernel": "gemm_tc_kernel",
+                    "achieved": 2.0 * R_mean * w.d * w.F / (launch_ms * 1e-3) / 1e12,
+                    "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
+            if w.dtype == "f32":
+                roof["bound"] = "alu"
+                roof["kernel"] = "gemm_simt_f32_kernel"
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["peak_source"] = f"{peak_src} ({'bf16_tflops_sustained' if roof['unit'] == 'TFLOP/s' else 'hbm_gbs'})"
+        roof["traffic"] = None
+        value = w.T * steps * world / (elapsed_ms * 1e-3)
+        cpu = None
+        if world == 1:
+            rate, n, dt = cpu_oracle_run(w, args.cpu_seconds)
+            cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                   "sample": f"first {n} tokens of one batch through the whole layer "
+                             f"({dt:.1f} s, capacity rescaled to the sample)"}
+        line = {"metric": "MoE layer tokens/s", "value": value, "unit": "tokens/s",
+                "n_gpus": world, "steps": steps, "warmup": warmup,
+                "ms_per_step": elapsed_ms / steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+                "config": config_of(w, world),
+                "e2e": {"value": w.T * e2e_steps * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": layer.launches_per_forward(gate=not w.logits_direct) * steps,
+                "roofline": roof, "stages": per, "clocks": clocks, "cpu_baseline": cpu,
+                "device_error_bits": dev_err}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,185 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE layer hot path.
+ *
+ * The layer, in the order the pages give it ("A Survey on Mixture of Experts",
+ * section 5 System Design: gate routing, input encode, expert computation,
+ * output decode; the All-to-All steps between them are the identity on one
+ * GPU):
+ *
+ *   moe_gate               router logits = x . Wg^T                     (a0)
+ *   moe_route              top-k softmax gate with expert capacity      (a1)
+ *   moe_dispatch           input encode: group each expert's tokens     (a2)
+ *   moe_expert_ffn         per-expert FC -> ReLU -> FC                  (a3)
+ *   moe_combine            output decode: gate-weighted un-permute      (a4)
+ *   moe_popularity_update  per-expert popularity, sliding-window mean   (a5)
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers to memory the caller owns.  The
+ *    library allocates nothing; the only scratch (moe_route's) is a caller
+ *    buffer sized by moe_route_workspace_size().
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and returns an int status: MOE_OK (0) or a negative
+ *    MOE_ERR_* code.  Arguments are validated on the host before anything is
+ *    launched; a call that returns an error has launched nothing.
+ *  - Row-major tensors, no padding between rows.  `dtype` is MOE_DTYPE_F32 or
+ *    MOE_DTYPE_BF16 (bf16 = the upper 16 bits of an IEEE binary32).
+ *  - Vector paths need every tensor base 16-byte aligned and every row a
+ *    multiple of 16 bytes (d, F multiples of 8 for bf16, of 4 for fp32);
+ *    anything else is rejected with MOE_ERR_UNSUPPORTED.
+ *  - Index tensors produced by moe_route are validated again on the device:
+ *    an out-of-range row index is skipped (never dereferenced) and recorded in
+ *    the per-device error word read by moe_device_error().
+ *  - Limits: 1 <= E <= 1024, 1 <= k <= min(E, 32), T*k < 2^31.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1, /* null pointer, size out of range, k > E, ...   */
+    MOE_ERR_UNSUPPORTED = -2, /* dtype or alignment the kernels do not handle */
+    MOE_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required   */
+    MOE_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed          */
+    MOE_ERR_DEVICE = -5       /* device-side check failed (moe_device_error)   */
+};
+
+enum moe_dtype { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+
+/* Device-side error bits (moe_device_error). */
+enum moe_device_error_bits {
+    MOE_DEVERR_ROW_INDEX = 1, /* a slot_row / row_slot entry outside [0, R_max) */
+    MOE_DEVERR_OFFSETS = 2,   /* offsets not non-decreasing or beyond R_max      */
+    MOE_DEVERR_TIMEOUT = 4    /* a pipeline wait inside a kernel ran past its
+                                 time limit; the kernel gave up and returned     */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(int status);
+
+/* Library ABI version: 100 * major + minor. */
+int moe_version(void);
+
+/* Reads the device error word of the CURRENT device (synchronous: waits for
+ * all work on the device) into *bits, then clears it if `clear` != 0.
+ * Returns MOE_OK or MOE_ERR_CUDA. */
+int moe_device_error(int32_t* bits, int clear);
+
+/* ---------------------------------------------------------------- a0 ----
+ * Router logits.  PopFetcher, section 2.1.2: the gate network scores each
+ * token against every expert.
+ *   x       [T, d]  dtype     tokens
+ *   Wg      [E, d]  dtype     one row per expert (out x in)
+ *   logits  [T, E]  fp32      logits[t][e] = sum_c x[t][c] * Wg[e][c],
+ *                             accumulated in fp32 (bf16 products are exact)
+ * T >= 0 (T = 0 launches nothing).  d >= 1.
+ */
+int moe_gate(const void* x, const void* Wg, int dtype, int T, int d, int E, float* logits,
+             moe_stream_t stream);
+
+/* ---------------------------------------------------------------- a1 ----
+ * Top-k softmax gate with GShard expert capacity.  "A Survey on Mixture of
+ * Experts", section 5 (gate routing; capacity-limited dispatch) and PopFetcher,
+ * section 2.1.2 (top-k gate); MoE-MPMC, problem statement (softmax router).
+ *
+ *   z[t][e] = logits[t][e] + bias[e]                (one fp32 addition)
+ *   ids[t][0..k-1]  the k largest z, larger first; equal z: lower index first
+ *   w[t][j]         = exp(z_j - z_0) / sum_{i<k} exp(z_i - z_0)  (fp32): the
+ *                     k softmax probabilities renormalised to sum to 1
+ *   counts[e]       tokens that chose e (demand, before drops)
+ *   kept[e]         min(counts[e], capacity)     (capacity <= 0: unlimited)
+ *   offsets[0..E]   exclusive prefix sum of kept; offsets[E] = R
+ *   slot_row[t][j]  row of slot (t, j) in the grouped layout, or -1 if dropped.
+ *                   Inside an expert, slots are ranked in token order; the
+ *                   first `capacity` are kept.
+ *   row_slot[r]     t*k + j of the slot stored in row r, for r < R.  The buffer
+ *                   must hold T*k entries; entries r >= R are not written.
+ *   n_dropped[0]    T*k - R
+ *
+ *   logits [T,E] fp32; bias [E] fp32 or NULL; ids, slot_row [T,k] int32;
+ *   w [T,k] fp32; counts, kept [E] int32; offsets [E+1] int32;
+ *   row_slot [T*k] int32; n_dropped [1] int32.
+ *   workspace: device buffer of at least moe_route_workspace_size(T, E, k)
+ *   bytes, 256-byte aligned; its contents need no initialisation.
+ * Results are bit-identical run to run (no atomics whose order is visible).
+ * T = 0 writes zeros to counts, kept, offsets and n_dropped.
+ */
+size_t moe_route_workspace_size(int T, int E, int k);
+
+int moe_route(const float* logits, const float* bias, int T, int E, int k, int capacity,
+              int32_t* ids, float* w, int32_t* counts, int32_t* kept, int32_t* offsets,
+              int32_t* slot_row, int32_t* row_slot, int32_t* n_dropped, void* workspace,
+              size_t workspace_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- a2 ----
+ * Input encode.  "A Survey on Mixture of Experts", section 5: the tokens
+ * routed to one expert are gathered into one contiguous block of rows.
+ *   Xp[slot_row[t][j]] = x[t]   for every kept slot (slot_row >= 0)
+ *   x [T, d] dtype; slot_row [T, k] from moe_route; Xp [R_max, d] dtype with
+ *   R_max >= R (T*k always suffices).  Rows of Xp that no slot names are left
+ *   untouched.  A slot_row entry >= R_max is skipped and flagged on the device.
+ */
+int moe_dispatch(const void* x, int dtype, int T, int d, int k, const int32_t* slot_row,
+                 void* Xp, int R_max, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- a3 ----
+ * Expert computation.  PopFetcher, section 5.1: each expert is FC(d -> F),
+ * ReLU, FC(F -> d) (two weight matrices, no bias terms).
+ *   for each expert e, rows r in [offsets[e], offsets[e+1]):
+ *     H[r][f]  = max(0, sum_c Xp[r][c] * W1[e][f][c])   stored in dtype
+ *     Yp[r][o] = sum_f H[r][f] * W2[e][o][f]             stored in dtype
+ *   Accumulation in fp32.  bf16 runs on the tcgen05 tensor cores; fp32 runs
+ *   on the CUDA cores (no TF32).
+ *   Xp [R_max, d]; W1 [E, F, d]; W2 [E, d, F]; offsets [E+1] (device, from
+ *   moe_route); H [R_max, F] caller scratch for the hidden activation;
+ *   Yp [R_max, d].  Rows >= offsets[E] of H and Yp are not written.
+ *   Offsets that decrease or exceed R_max are flagged on the device and the
+ *   offending expert is skipped.
+ */
+int moe_expert_ffn(const void* Xp, const void* W1, const void* W2, int dtype, int E, int d,
+                   int F, const int32_t* offsets, int R_max, void* H, void* Yp,
+                   moe_stream_t stream);
+
+/* ---------------------------------------------------------------- a4 ----
+ * Output decode.  "A Survey on Mixture of Experts", section 5: the inverse of
+ * input encode restores token order by the gating indices; each token's
+ * output is the gate-weighted sum of its experts' outputs:
+ *   y[t] = sum_{j < k, slot_row[t][j] >= 0} w[t][j] * Yp[slot_row[t][j]]
+ *   accumulated in fp32 with j ascending, rounded once to dtype.  A token
+ *   whose slots were all dropped gets zeros.
+ *   Yp [R_max, d] dtype; slot_row, w [T, k]; y [T, d] dtype.
+ */
+int moe_combine(const void* Yp, int dtype, int T, int d, int k, const int32_t* slot_row,
+                const float* w, void* y, int R_max, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- a5 ----
+ * Expert popularity over a sliding window.  PopFetcher, section 3.1 (the
+ * routing information collector counts the tokens routed to each expert) and
+ * section 4.2 (Eq. 1, a window over recent iterations; read here as the
+ * arithmetic mean of the last n = min(step + 1, W) count vectors).
+ *   hist [W, E] int32   caller-owned ring; step `step` writes row step % W.
+ *                       Start from any contents at step 0: rows not yet
+ *                       written are never read.
+ *   mean [E] fp32       (float)window_sum / (float)n, correctly rounded
+ *   hot  [P] int32      the P experts with the largest window sum, larger
+ *                       first, equal sums to the lower index
+ *   counts [E] int32 (e.g. moe_route's); 0 <= P <= E; W >= 1; step >= 0.
+ *   The state across steps is hist plus the caller's step counter: copying
+ *   hist out and back resumes the sequence exactly.
+ */
+int moe_popularity_update(const int32_t* counts, int E, int32_t* hist, int W, int64_t step,
+                          float* mean, int P, int32_t* hot, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,68 @@
+// common.cuh -- helpers shared by the MoE kernels (device side and host-side
+// argument checks).  Nothing here is shared with the CPU oracle.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 32;
+
+// Per-device error word (defined in abi.cu): device-side checks OR bits into
+// it instead of faulting; moe_device_error() reads and clears it.  Kernels in
+// other translation units receive its address as an argument.
+int32_t* device_error_word();  // nullptr if the symbol lookup failed
+
+__device__ __forceinline__ void flag_error(int32_t* err, int32_t bits) {
+    if (err) atomicOr(err, bits);
+}
+
+// ----------------------------------------------------------------- host ----
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t dtype_bytes(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2u : 4u; }
+inline bool dtype_ok(int dtype) { return dtype == MOE_DTYPE_F32 || dtype == MOE_DTYPE_BF16; }
+
+// Launch-error check: returns MOE_ERR_CUDA if the last launch failed.
+inline int launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+inline int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+// --------------------------------------------------------------- device ----
+// 16-byte global accesses.  Loads of read-only inputs bypass L1 allocation.
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void stg_v4(void* p, const uint4& v) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// Two floats -> packed bf16x2 (round to nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+}  // namespace moe

@@ -1,0 +1,456 @@
+// gemm_tc.cu -- grouped bf16 GEMM on the 5th-generation tensor cores.
+//
+// Expert computation (PopFetcher, section 5.1: FC(d -> F), ReLU, FC(F -> d))
+// over the contiguous per-expert row blocks of input encode ("A Survey on
+// Mixture of Experts", section 5), and the gate projection as one group.
+//
+//   C[r][n] = act( sum_k A[r][k] * B_e[n][k] )   r in group e, fp32 accumulate
+//
+// A [R_max, K] and B [E*N, K] are bf16, K-major.  One persistent CTA per SM
+// walks a static round-robin over the device-built tile table (grouped.cuh).
+// Warp roles (192 threads):
+//   warp 0     one lane issues TMA loads of 128x64 A and BNx64 B tiles (128-byte
+//              swizzle) into a kStages-deep shared-memory ring;
+//   warp 1     allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN, K=16,
+//              kind::f16, bf16 in, fp32 accumulate in TMEM) and tcgen05.commit
+//              to free ring slots and publish finished accumulators;
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator (one row per thread,
+//              lane quadrant = warp % 4), ReLU, round to bf16 (or keep fp32),
+//              row-masked 16-byte stores (rows past the group end belong to
+//              the next group and are never written).
+// Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap the
+// mainloop of tile i+1.  Every mbarrier wait is bounded in time: on expiry the
+// kernel flags MOE_DEVERR_TIMEOUT, drains its own TMA loads and MMAs, frees
+// TMEM and returns.
+#include <cuda.h>
+
+#include "grouped.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // one 128-byte swizzle row of bf16
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
+
+template <int BN>
+struct Cfg {
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64
+                                   : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+    // ring + barriers/flags (256 B) + warp scratch (128 B) + tile prefix + alignment slack
+    static constexpr int fixed_bytes() { return kStages * STAGE_BYTES + 256 + 128 + 1024; }
+    static int smem_bytes(int E) { return fixed_bytes() + 4 * (E + 1); }
+};
+
+// ------------------------------------------------------------ PTX wrappers --
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Waits for the phase of `bar` with the given parity.  Gives up (returns
+// false) when another role has raised the abort flag, or after kTimeoutNs, in
+// which case it raises the flag and records MOE_DEVERR_TIMEOUT.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                       int32_t* err, bool honour_abort = true) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait(a, parity)) return true;
+        if ((spin & 63u) == 0) {
+            if (honour_abort && *abort_flag) return false;
+            if (globaltimer() - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                flag_error(err, MOE_DEVERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+// Shared-memory matrix descriptor: K-major tile whose rows are 128 bytes with
+// the 128-byte swizzle, 8-row core groups 1024 bytes apart (tile base must be
+// 1024-byte aligned; +32 bytes steps one K=16 slice inside the swizzle row).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address
+    d |= static_cast<uint64_t>(1) << 16;                  // leading byte offset (unused here)
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;          // stride byte offset
+    d |= static_cast<uint64_t>(1) << 46;                  // descriptor version
+    d |= static_cast<uint64_t>(2) << 61;                  // 128-byte swizzle
+    return d;
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ epilogue
+template <typename TOut, bool RELU>
+struct Store32;
+template <bool RELU>
+struct Store32<__nv_bfloat16, RELU> {
+    // 32 consecutive columns of one row; N % 8 == 0 is guaranteed by the host.
+    __device__ static void run(__nv_bfloat16* dst, const uint32_t (&r)[32], int cols_left) {
+        uint32_t p[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float lo = __uint_as_float(r[2 * i]), hi = __uint_as_float(r[2 * i + 1]);
+            if (RELU) {
+                lo = lo > 0.0f ? lo : 0.0f;
+                hi = hi > 0.0f ? hi : 0.0f;
+            }
+            p[i] = pack_bf16x2(lo, hi);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (q * 8 < cols_left)
+                stg_v4(dst + q * 8, make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]));
+    }
+};
+template <bool RELU>
+struct Store32<float, RELU> {
+    __device__ static void run(float* dst, const uint32_t (&r)[32], int cols_left) {
+        if (cols_left >= 32 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                uint4 v = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+                if (RELU) {
+                    v.x = __float_as_uint(fmaxf(__uint_as_float(v.x), 0.0f));
+                    v.y = __float_as_uint(fmaxf(__uint_as_float(v.y), 0.0f));
+                    v.z = __float_as_uint(fmaxf(__uint_as_float(v.z), 0.0f));
+                    v.w = __float_as_uint(fmaxf(__uint_as_float(v.w), 0.0f));
+                }
+                stg_v4(dst + 4 * q, v);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (i < cols_left) {
+                    const float v = __uint_as_float(r[i]);
+                    dst[i] = RELU ? (v > 0.0f ? v : 0.0f) : v;
+                }
+            }
+        }
+    }
+};
+
+// -------------------------------------------------------------------- kernel
+template <int BN, bool RELU, typename TOut>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+               TOut* __restrict__ C, int N, int K, int E, const int32_t* __restrict__ offsets,
+               int single_M, int R_max, int32_t* err) {
+    using G = Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~static_cast<uintptr_t>(1023u));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * G::A_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * G::B_BYTES);
+    uint64_t* full = bars;               // [kStages] TMA -> MMA
+    uint64_t* empty = bars + kStages;    // [kStages] MMA -> TMA
+    uint64_t* tfull = empty + kStages;   // [2] MMA -> epilogue
+    uint64_t* tempty = tfull + 2;        // [2] epilogue -> MMA
+    uint64_t* drain = tempty + 2;        // [1] final MMA completion
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int32_t* s_warp = reinterpret_cast<int32_t*>(bars) + 64;  // 256 B past the barriers
+    int32_t* s_prefix = s_warp + 32;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull + a, 1);
+            mbar_init(tempty + a, kEpiThreads);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, G::TMEM_COLS);
+        tmem_relinquish();
+    }
+    const int nt = (N + BN - 1) / BN;
+    const int total = build_tile_table(offsets, single_M, E, nt, BM, R_max, s_prefix, s_warp, err);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int nk = (K + BK - 1) / BK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)));
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)));
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                const TileCoord c = tile_coord(tile, s_prefix, E, offsets, single_M, BM, BN);
+                const int b_row = c.e * N + c.n0;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(full + stage, G::STAGE_BYTES);
+                    tma_load_2d(sA + stage * G::A_BYTES, &tmap_a, full + stage, kb * BK, c.row0);
+                    tma_load_2d(sB + stage * G::B_BYTES, &tmap_b, full + stage, kb * BK, b_row);
+                    ++issued;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // Let the loads already issued land before the CTA exits.
+                const long long n = issued < kStages ? issued : kStages;
+                for (long long i = issued - n; i < issued; ++i)
+                    mbar_wait(full + (int)(i % kStages), (uint32_t)((i / kStages) & 1), abort_flag,
+                              err, false);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = idesc_bf16(BM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int it = 0;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
+                const int acc = it & 1;
+                if (!mbar_wait(tempty + acc, ((it >> 1) & 1) ^ 1u, abort_flag, err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(full + stage, phase, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * G::A_BYTES);
+                    const uint32_t b0 = smem_u32(sB + stage * G::B_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_bf16(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc,
+                                 (kb | kk) != 0 ? 1u : 0u);
+                    mma_commit(empty + stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) mma_commit(tfull + acc);
+            }
+            // all MMAs this thread issued are complete once `drain` fires
+            mma_commit(drain);
+            mbar_wait(drain, 0, abort_flag, err, false);
+        }
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+            const TileCoord c = tile_coord(tile, s_prefix, E, offsets, single_M, BM, BN);
+            const int acc = it & 1;
+            if (!mbar_wait(tfull + acc, (it >> 1) & 1, abort_flag, err)) break;
+            tc_fence_after();
+            const bool row_ok = row < c.rows;
+            TOut* crow = C + static_cast<size_t>(c.row0 + (row_ok ? row : 0)) * N;
+#pragma unroll 1
+            for (int cc = 0; cc < BN; cc += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + cc), r);
+                const int col = c.n0 + cc;
+                if (row_ok && col < N) Store32<TOut, RELU>::run(crow + col, r, N - col);
+            }
+            tc_fence_before();
+            mbar_arrive(tempty + acc);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, G::TMEM_COLS);
+    }
+}
+
+// -------------------------------------------------------------------- host --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (inner contiguous), box [box_outer, 64].
+static int make_tmap(CUtensorMap* m, const void* base, int inner, int outer, int box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return MOE_ERR_CUDA;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_outer)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <int BN, bool RELU, typename TOut>
+static int launch(const void* A, const void* B, TOut* C, int N, int K, int E,
+                  const int32_t* offsets, int single_M, int R_max, cudaStream_t st) {
+    using G = Cfg<BN>;
+    if (R_max <= 0 || N <= 0) return MOE_OK;
+    CUtensorMap ta, tb;
+    if (make_tmap(&ta, A, K, R_max, BM) != MOE_OK) return MOE_ERR_CUDA;
+    if (make_tmap(&tb, B, K, E * N, BN) != MOE_OK) return MOE_ERR_CUDA;
+    const int smem = G::smem_bytes(E);
+    auto kern = gemm_tc_kernel<BN, RELU, TOut>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const int nt = (N + BN - 1) / BN;
+    const long long ub = ((long long)R_max / BM + E) * nt;
+    const int grid = (int)(ub < num_sms() ? ub : num_sms());
+    kern<<<grid, kThreads, smem, st>>>(ta, tb, C, N, K, E, offsets, single_M, R_max,
+                                       device_error_word());
+    return launch_status();
+}
+
+}  // namespace tc
+
+int launch_gemm_tc_bf16(const void* A, const void* B, void* C, bool out_f32, int N, int K, int E,
+                        const int32_t* offsets, int single_M, int R_max, bool relu,
+                        cudaStream_t st) {
+    using namespace tc;
+    if (out_f32) {
+        float* Cf = static_cast<float*>(C);
+        if (relu) return MOE_ERR_UNSUPPORTED;
+        if (N <= 32) return launch<32, false, float>(A, B, Cf, N, K, E, offsets, single_M, R_max, st);
+        if (N <= 64) return launch<64, false, float>(A, B, Cf, N, K, E, offsets, single_M, R_max, st);
+        if (N <= 128) return launch<128, false, float>(A, B, Cf, N, K, E, offsets, single_M, R_max, st);
+        return launch<256, false, float>(A, B, Cf, N, K, E, offsets, single_M, R_max, st);
+    }
+    __nv_bfloat16* Cb = static_cast<__nv_bfloat16*>(C);
+    if (relu) return launch<256, true, __nv_bfloat16>(A, B, Cb, N, K, E, offsets, single_M, R_max, st);
+    return launch<256, false, __nv_bfloat16>(A, B, Cb, N, K, E, offsets, single_M, R_max, st);
+}
+
+}  // namespace moe

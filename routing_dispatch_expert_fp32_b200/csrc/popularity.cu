@@ -1,0 +1,58 @@
+// popularity.cu -- moe_popularity_update: per-expert popularity over a
+// sliding window of steps.
+//
+// PopFetcher, section 3.1: the routing information collector counts the tokens
+// routed to each expert (the expert's popularity).  Section 4.2, Eq. 1 (lost in
+// extraction): popularity is averaged over a window of recent iterations.
+// Reading taken: mean of the last n = min(step + 1, W) count vectors; hot
+// experts ranked by window sum (desc), equal sums to the lower index.
+//
+// One CTA: thread e writes this step's count into ring row step % W, sums its
+// column over the n live rows (int64), writes the correctly rounded mean, and
+// ranks itself against every other expert's sum (E <= 1024, O(E^2 / threads)).
+#include "common.cuh"
+
+namespace moe {
+
+__global__ void __launch_bounds__(1024)
+popularity_kernel(const int32_t* __restrict__ counts, int E, int32_t* __restrict__ hist, int W,
+                  long long step, float* __restrict__ mean, int P, int32_t* __restrict__ hot) {
+    __shared__ long long s_sum[kMaxExperts];
+    const int slot = (int)(step % W);
+    const long long n = step + 1 < W ? step + 1 : W;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int32_t c = counts[e];
+        hist[(size_t)slot * E + e] = c;
+        long long sum = c;
+        for (long long i = 1; i < n; ++i) {
+            const int s = (int)((step - i) % W);
+            sum += hist[(size_t)s * E + e];
+        }
+        s_sum[e] = sum;
+        mean[e] = __fdiv_rn(__ll2float_rn(sum), __ll2float_rn(n));
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const long long mine = s_sum[e];
+        int rank = 0;
+        for (int o = 0; o < E; ++o) {
+            const long long v = s_sum[o];
+            rank += (v > mine) || (v == mine && o < e);
+        }
+        if (rank < P) hot[rank] = e;
+    }
+}
+
+}  // namespace moe
+
+extern "C" int moe_popularity_update(const int32_t* counts, int E, int32_t* hist, int W,
+                                     int64_t step, float* mean, int P, int32_t* hot,
+                                     moe_stream_t stream) {
+    using namespace moe;
+    if (E < 1 || E > kMaxExperts || W < 1 || step < 0 || P < 0 || P > E) return MOE_ERR_INVALID_ARG;
+    if (!counts || !hist || !mean || (P > 0 && !hot)) return MOE_ERR_INVALID_ARG;
+    const int threads = ((E + 31) / 32) * 32;
+    popularity_kernel<<<1, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        counts, E, hist, W, (long long)step, mean, P, hot);
+    return launch_status();
+}

@@ -1,0 +1,192 @@
+"""ctypes binding of libmoe.so (include/moe.h): argument marshalling only.
+
+Every function has the C name, takes torch tensors that live on the current
+CUDA device, passes their data pointers and the current stream, and raises
+MoeError on a non-zero status.  Every step of the computation runs in the
+library's CUDA kernels; there is no other implementation behind these names.
+If libmoe.so is missing this module fails to import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                      "`python -m routing_dispatch_expert_fp32_b200.build` (needs nvcc)")
+lib = ctypes.CDLL(_LIB_PATH)
+
+MOE_OK = 0
+MOE_DTYPE_F32 = 0
+MOE_DTYPE_BF16 = 1
+MOE_DEVERR_ROW_INDEX = 1
+MOE_DEVERR_OFFSETS = 2
+MOE_DEVERR_TIMEOUT = 4
+
+_p, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+_SIGS = {
+    "moe_status_string": ([_i], ctypes.c_char_p),
+    "moe_version": ([], _i),
+    "moe_device_error": ([_p, _i], _i),
+    "moe_gate": ([_p, _p, _i, _i, _i, _i, _p, _p], _i),
+    "moe_route_workspace_size": ([_i, _i, _i], _sz),
+    "moe_route": ([_p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p], _i),
+    "moe_dispatch": ([_p, _i, _i, _i, _i, _p, _p, _i, _p], _i),
+    "moe_expert_ffn": ([_p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _p, _p], _i),
+    "moe_combine": ([_p, _i, _i, _i, _i, _p, _p, _p, _i, _p], _i),
+    "moe_popularity_update": ([_p, _i, _p, _i, _i64, _p, _i, _p, _p], _i),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes, _f.restype = _args, _res
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = lib.moe_status_string(status).decode()
+        super().__init__(f"{fn} failed: {msg} ({status})")
+        self.status = status
+
+
+def _check(fn: str, status: int) -> None:
+    if status != MOE_OK:
+        raise MoeError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MOE_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return MOE_DTYPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def moe_version() -> int:
+    return lib.moe_version()
+
+
+def moe_device_error(clear: bool = True) -> int:
+    bits = ctypes.c_int32(0)
+    _check("moe_device_error", lib.moe_device_error(ctypes.byref(bits), int(clear)))
+    return bits.value
+
+
+def moe_gate(x, Wg, logits, stream=None):
+    T, d = x.shape
+    E = Wg.shape[0]
+    _check("moe_gate", lib.moe_gate(_ptr(x), _ptr(Wg), dtype_code(x), T, d, E, _ptr(logits),
+                                     _stream(stream)))
+
+
+def moe_route_workspace_size(T: int, E: int, k: int) -> int:
+    return int(lib.moe_route_workspace_size(T, E, k))
+
+
+def moe_route(logits, bias, k, capacity, ids, w, counts, kept, offsets, slot_row, row_slot,
+              n_dropped, workspace, stream=None):
+    T, E = logits.shape
+    _check("moe_route", lib.moe_route(
+        _ptr(logits), _ptr(bias), T, E, k, int(capacity), _ptr(ids), _ptr(w), _ptr(counts),
+        _ptr(kept), _ptr(offsets), _ptr(slot_row), _ptr(row_slot), _ptr(n_dropped),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_dispatch(x, k, slot_row, Xp, stream=None):
+    T, d = x.shape
+    _check("moe_dispatch", lib.moe_dispatch(_ptr(x), dtype_code(x), T, d, k, _ptr(slot_row),
+                                            _ptr(Xp), Xp.shape[0], _stream(stream)))
+
+
+def moe_expert_ffn(Xp, W1, W2, offsets, H, Yp, stream=None):
+    E, F, d = W1.shape
+    _check("moe_expert_ffn", lib.moe_expert_ffn(
+        _ptr(Xp), _ptr(W1), _ptr(W2), dtype_code(Xp), E, d, F, _ptr(offsets), Xp.shape[0],
+        _ptr(H), _ptr(Yp), _stream(stream)))
+
+
+def moe_combine(Yp, k, slot_row, w, y, stream=None):
+    T, d = y.shape
+    _check("moe_combine", lib.moe_combine(_ptr(Yp), dtype_code(Yp), T, d, k, _ptr(slot_row),
+                                          _ptr(w), _ptr(y), Yp.shape[0], _stream(stream)))
+
+
+def moe_popularity_update(counts, hist, step, mean, P, hot, stream=None):
+    W, E = hist.shape
+    _check("moe_popularity_update", lib.moe_popularity_update(
+        _ptr(counts), E, _ptr(hist), W, int(step), _ptr(mean), P, _ptr(hot), _stream(stream)))
+
+
+class MoELayer:
+    """One MoE layer's device buffers plus the call sequence of the hot path.
+
+    Weights stay resident; ``forward`` runs gate (unless logits are given),
+    route, popularity, dispatch, expert FFN and combine on the current stream,
+    all through the C ABI.  ``identity_experts`` skips the FFN (Yp = Xp).
+    """
+
+    def __init__(self, T, d, E, k, F, dtype, capacity=0, W=4, P=8, device="cuda",
+                 identity_experts=False):
+        self.T, self.d, self.E, self.k, self.F = T, d, E, k, F
+        self.dtype, self.capacity, self.W, self.P = dtype, capacity, W, P
+        self.identity_experts = identity_experts
+        dev, i32 = device, torch.int32
+        Rmax = max(T * k, 1)
+        self.logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+        self.ids = torch.empty(T, k, dtype=i32, device=dev)
+        self.w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.counts = torch.empty(E, dtype=i32, device=dev)
+        self.kept = torch.empty(E, dtype=i32, device=dev)
+        self.offsets = torch.empty(E + 1, dtype=i32, device=dev)
+        self.slot_row = torch.empty(T, k, dtype=i32, device=dev)
+        self.row_slot = torch.empty(Rmax, dtype=i32, device=dev)
+        self.n_dropped = torch.empty(1, dtype=i32, device=dev)
+        self.workspace = torch.empty(moe_route_workspace_size(T, E, k), dtype=torch.uint8,
+                                     device=dev)
+        self.Xp = torch.empty(Rmax, d, dtype=dtype, device=dev)
+        self.H = None if identity_experts else torch.empty(Rmax, F, dtype=dtype, device=dev)
+        self.Yp = self.Xp if identity_experts else torch.empty(Rmax, d, dtype=dtype, device=dev)
+        self.y = torch.empty(T, d, dtype=dtype, device=dev)
+        self.hist = torch.zeros(W, E, dtype=i32, device=dev)
+        self.mean = torch.empty(E, dtype=torch.float32, device=dev)
+        self.hot = torch.empty(max(P, 1), dtype=i32, device=dev)
+        self.step = 0
+
+    def forward(self, x, Wg=None, W1=None, W2=None, bias=None, logits=None, stream=None,
+                popularity=True, counts_hook=None):
+        if logits is None:
+            moe_gate(x, Wg, self.logits, stream)
+            logits = self.logits
+        moe_route(logits, bias, self.k, self.capacity, self.ids, self.w, self.counts, self.kept,
+                  self.offsets, self.slot_row, self.row_slot, self.n_dropped, self.workspace,
+                  stream)
+        if popularity:
+            if counts_hook is not None:  # e.g. an all_reduce of the counts across ranks
+                counts_hook(self.counts)
+            moe_popularity_update(self.counts, self.hist, self.step, self.mean, self.P, self.hot,
+                                  stream)
+            self.step += 1
+        moe_dispatch(x, self.k, self.slot_row, self.Xp, stream)
+        if not self.identity_experts:
+            moe_expert_ffn(self.Xp, W1, W2, self.offsets, self.H, self.Yp, stream)
+        moe_combine(self.Yp, self.k, self.slot_row, self.w, self.y, stream)
+        return self.y
+
+    def launches_per_forward(self, gate=True, popularity=True) -> int:
+        """Kernel launches one forward makes (route is three kernels)."""
+        n = 3 + 1 + 1  # route, dispatch, combine
+        n += 1 if gate else 0
+        n += 1 if popularity else 0
+        n += 0 if self.identity_experts else 2
+        return n

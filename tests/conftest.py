@@ -13,3 +13,17 @@ def pytest_configure(config):
 
 
 GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(scope="session")
+def libmoe_path():
+    """Builds libmoe.so in-tree if it is missing or older than its sources."""
+    from routing_dispatch_expert_fp32_b200 import build
+    return build.build()
+
+
+@pytest.fixture(scope="session")
+def moe(libmoe_path):
+    """The ctypes binding (GPU tests only call compute entry points)."""
+    from routing_dispatch_expert_fp32_b200 import moe as m
+    return m

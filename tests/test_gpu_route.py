@@ -1,0 +1,118 @@
+"""moe_route on the GPU against the oracle: bit-exact ids, counts, kept,
+offsets, slot_row, row_slot, n_dropped; weights within fp32 rounding."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import dev, host
+from routing_dispatch_expert_fp32_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def run_route(moe, logits, bias, k, capacity):
+    T, E = logits.shape
+    i32 = torch.int32
+    L = dev(logits)
+    B = None if bias is None else dev(bias)
+    out = dict(ids=torch.full((T, k), -7, dtype=i32, device="cuda"),
+               w=torch.full((T, k), -7.0, device="cuda"),
+               counts=torch.full((E,), -7, dtype=i32, device="cuda"),
+               kept=torch.full((E,), -7, dtype=i32, device="cuda"),
+               offsets=torch.full((E + 1,), -7, dtype=i32, device="cuda"),
+               slot_row=torch.full((T, k), -7, dtype=i32, device="cuda"),
+               row_slot=torch.full((max(T * k, 1),), -7, dtype=i32, device="cuda"),
+               n_dropped=torch.full((1,), -7, dtype=i32, device="cuda"))
+    ws = torch.empty(moe.moe_route_workspace_size(T, E, k), dtype=torch.uint8, device="cuda")
+    moe.moe_route(L, B, k, capacity, out["ids"], out["w"], out["counts"], out["kept"],
+                  out["offsets"], out["slot_row"], out["row_slot"], out["n_dropped"], ws)
+    torch.cuda.synchronize()
+    return {n: host(t) for n, t in out.items()}
+
+
+def check_route(moe, logits, bias, k, capacity):
+    g = run_route(moe, logits, bias, k, capacity)
+    r = oracle.route(logits, bias, k, capacity)
+    R = int(r["offsets"][-1])
+    for name in ["ids", "counts", "kept", "offsets", "slot_row"]:
+        assert np.array_equal(g[name], r[name]), name
+    assert np.array_equal(g["row_slot"][:R], r["row_slot"]), "row_slot"
+    assert int(g["n_dropped"][0]) == r["n_dropped"]
+    np.testing.assert_allclose(g["w"], r["w"], rtol=4e-6, atol=1e-8)
+    if logits.shape[0]:
+        np.testing.assert_allclose(g["w"].astype(np.float64).sum(1), 1.0, atol=2e-6)
+    assert moe.moe_device_error() == 0
+    return g, r
+
+
+WORKLOAD_SHAPES = [  # (T, E, k, capacity, zipf_s) of the five layer workloads
+    (512, 8, 2, 0, None), (4096, 16, 2, 640, 1.2), (16384, 64, 2, 640, 1.1),
+    (32768, 256, 8, 0, 1.0), (65536, 128, 4, 0, None), (65536, 128, 4, 0, 1.5),
+]
+
+
+@pytest.mark.parametrize("T,E,k,cap,s", WORKLOAD_SHAPES)
+def test_route_workload_shapes(moe, T, E, k, cap, s):
+    w = wl.tiny("r", T=T, d=8, E=E, k=k, F=8, zipf_s=s, capacity_factor=None, index=50 + E)
+    rng = wl.rng_for(w, 0, wl.TENSOR_LOGITS)
+    logits = rng.standard_normal((T, E), dtype=np.float32)
+    check_route(moe, logits, wl.zipf_bias(w), k, cap)
+
+
+@pytest.mark.parametrize("T,E,k,cap", [
+    (1, 4, 2, 0), (1, 1, 1, 0), (7, 3, 3, 0), (129, 5, 5, 2), (200, 12, 3, 7), (257, 100, 7, 3),
+    (300, 33, 4, 0), (1000, 1024, 32, 0), (513, 1000, 8, 1), (130, 17, 16, 0), (4097, 9, 1, 100),
+])
+def test_route_edge_shapes(moe, T, E, k, cap):
+    rng = np.random.default_rng(T * 7 + E)
+    logits = rng.standard_normal((T, E), dtype=np.float32)
+    bias = rng.standard_normal(E).astype(np.float32)
+    check_route(moe, logits, bias, k, cap)
+
+
+def test_route_ties_break_to_lower_index(moe):
+    rng = np.random.default_rng(3)
+    logits = rng.integers(-2, 3, (777, 24)).astype(np.float32)  # many exact ties
+    logits[5] = 0.0
+    logits[6, ::2] = -0.0
+    check_route(moe, logits, None, 5, 40)
+
+
+def test_route_all_tokens_to_one_expert(moe):
+    T, E = 1000, 16
+    logits = np.tile(np.linspace(-1, 1, E, dtype=np.float32)[::-1], (T, 1))
+    g, r = check_route(moe, logits, None, 2, 100)
+    assert g["counts"][0] == T and g["kept"][0] == 100 and g["n_dropped"][0] == 2 * T - 200
+
+
+def test_route_capacity_zero_means_unlimited_and_capacity_one(moe):
+    rng = np.random.default_rng(4)
+    logits = rng.standard_normal((640, 16), dtype=np.float32)
+    check_route(moe, logits, None, 2, 0)
+    g, _ = check_route(moe, logits, None, 2, 1)
+    assert g["kept"].max() == 1
+
+
+def test_route_golden_example(moe):
+    import json, os
+    from conftest import GOLDEN
+    gd = json.load(open(os.path.join(GOLDEN, "route_example_a.json")))
+    g, _ = check_route(moe, np.array(gd["logits"], np.float32), None, gd["k"], gd["capacity"])
+    assert g["slot_row"].tolist() == gd["slot_row"]
+    assert g["row_slot"][:7].tolist() == gd["row_slot"]
+
+
+def test_route_empty_batch(moe):
+    g = run_route(moe, np.zeros((0, 8), np.float32), None, 2, 0)
+    assert g["counts"].tolist() == [0] * 8 and g["offsets"].tolist() == [0] * 9
+    assert g["n_dropped"][0] == 0
+
+
+def test_route_is_deterministic(moe):
+    rng = np.random.default_rng(5)
+    logits = rng.standard_normal((20000, 64), dtype=np.float32)
+    runs = [run_route(moe, logits, None, 4, 900) for _ in range(3)]
+    for other in runs[1:]:
+        for name in runs[0]:
+            assert np.array_equal(runs[0][name], other[name]), name
