@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--no-bias", action="store_true", help="bw_sweep without the Zipf bias")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
-                    help="target CPU time of the oracle sample")
+                    help="target CPU time of the oracle sample (0: skip the CPU leg)")
     return ap.parse_args()
 
 
@@ -400,7 +400,7 @@ def main():
         roof["traffic"] = None
         value = w.T * steps * world / (elapsed_ms * 1e-3)
         cpu = None
-        if world == 1:
+        if world == 1 and args.cpu_seconds > 0:
             rate, n, dt = cpu_oracle_run(w, args.cpu_seconds)
             cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                    "sample": f"first {n} tokens of one batch through the whole layer "
