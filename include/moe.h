@@ -119,6 +119,30 @@ int moe_route(const float* logits, const float* bias, int T, int E, int k, int c
               int32_t* slot_row, int32_t* row_slot, int32_t* n_dropped, void* workspace,
               size_t workspace_bytes, moe_stream_t stream);
 
+/* moe_route without a caller workspace (the pages have no counterpart; this
+ * is an integration convenience).  For callers that may not allocate device
+ * memory where they run the layer (fixed memory plans in serving loops,
+ * plugins whose host framework owns all allocations, code that must avoid
+ * the device-wide synchronisation an allocation can trigger).  Same arguments,
+ * results and errors as moe_route, minus the workspace: the scratch is a
+ * 4 MiB device array built into the library (held on every device that loads
+ * it until the process exits).
+ *  - Size limit: moe_route_workspace_size(T, E, k) <= 4 MiB (e.g. E = 256 up
+ *    to T = 262144 tokens, E = 1024 up to T = 65536); larger problems return
+ *    MOE_ERR_WORKSPACE and launch nothing.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls share the one array: calls whose kernels may overlap on a
+ *    device (several streams or host threads) race and must be serialised by
+ *    the caller.  Nothing in it needs clearing between calls.
+ *  - Allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
+ */
+int moe_route_noalloc(const float* logits, const float* bias, int T, int E, int k, int capacity,
+                      int32_t* ids, float* w, int32_t* counts, int32_t* kept, int32_t* offsets,
+                      int32_t* slot_row, int32_t* row_slot, int32_t* n_dropped,
+                      moe_stream_t stream);
+
 /* ---------------------------------------------------------------- a2 ----
  * Input encode.  "A Survey on Mixture of Experts", section 5: the tokens
  * routed to one expert are gathered into one contiguous block of rows.

@@ -294,3 +294,83 @@ extern "C" int moe_route(const float* logits, const float* bias, int T, int E, i
     }
     return MOE_OK;
 }
+
+// ------------------------------------------------------------------------
+// moe_route_noalloc: moe_route for callers that cannot allocate device memory.
+//
+// Some callers are not allowed to allocate on the path that runs the layer:
+// serving loops with a fixed memory plan, plugins inside a host framework that
+// owns every device allocation, code that must not risk the implicit device
+// synchronisation cudaMalloc/cudaFree can cause.  For them the router's scratch
+// (per-chunk histograms and bases) lives in a fixed device array compiled into
+// this library, so the call needs nothing beyond its inputs and outputs.
+//
+// The array below is a host-side placeholder symbol in host code, not a device
+// address.  Its device address is looked up once per device with
+// cudaGetSymbolAddress, with that device current, the first time the entry
+// point runs there; that first call should therefore happen before any stream
+// capture.  Every call shares the one array: two calls whose kernels overlap on
+// the device (different streams, or different host threads) race on it and
+// must be serialised by the caller.  The router's kernels overwrite every
+// scratch word they read, so nothing has to be cleared between calls.
+namespace moe {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB on every device
+static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
+
+static void* noalloc_scratch_ptr() {
+    constexpr int kMaxDevices = 64;
+    static void* cache[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
+        cache[dev] = p;
+    }
+    return cache[dev];
+}
+
+}  // namespace moe
+
+extern "C" int moe_route_noalloc(const float* logits, const float* bias, int T, int E, int k,
+                                 int capacity, int32_t* ids, float* w, int32_t* counts,
+                                 int32_t* kept, int32_t* offsets, int32_t* slot_row,
+                                 int32_t* row_slot, int32_t* n_dropped, moe_stream_t stream) {
+    if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > kMaxTopK)
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)T * k >= INT32_MAX) return MOE_ERR_INVALID_ARG;
+    if (!counts || !kept || !offsets || !n_dropped) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !ids || !w || !slot_row || !row_slot)) return MOE_ERR_INVALID_ARG;
+    // The fixed scratch bounds the problem size.
+    if (moe_route_workspace_size(T, E, k) > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
+    void* scratch = noalloc_scratch_ptr();
+    if (!scratch) return MOE_ERR_CUDA;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    char* ws = static_cast<char*>(scratch);  // 256-byte aligned by declaration
+    int32_t* hist = reinterpret_cast<int32_t*>(ws);
+    int32_t* base = reinterpret_cast<int32_t*>(ws + align256((size_t)nchunks * E * 4));
+
+    if (T > 0) {
+        if (E <= 8) launch_topk<8, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 16) launch_topk<16, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 32) launch_topk<32, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 64) launch_topk<32, 2>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 128) launch_topk<32, 4>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 256) launch_topk<32, 8>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 512) launch_topk<32, 16>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else launch_topk<32, 32>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
+    }
+    route_scan_kernel<<<1, kScanThreads, 0, st>>>(hist, nchunks, T, E, k, capacity, base, counts,
+                                                  kept, offsets, n_dropped);
+    if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
+    if (T > 0) {
+        route_assign_kernel<<<nchunks, kThreads, 0, st>>>(ids, T, E, k, capacity, base, offsets,
+                                                          slot_row, row_slot);
+        if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
