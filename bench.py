@@ -47,7 +47,11 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--tokens", type=int, default=0, help="override T (bw_sweep sizes)")
     ap.add_argument("--no-bias", action="store_true", help="bw_sweep without the Zipf bias")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override E (smaller profiling cases of the same shapes)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-graph", action="store_true",
+                    help="issue the step kernel by kernel instead of replaying a CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample (0: skip the CPU leg)")
     return ap.parse_args()
@@ -59,6 +63,8 @@ def workload_of(args) -> wl.Workload:
         w = w.with_(T=args.tokens)
     if args.no_bias:
         w = w.with_(zipf_s=None)
+    if args.experts:
+        w = w.with_(E=args.experts)
     return w
 
 
@@ -263,9 +269,8 @@ def main():
                       layer.n_dropped, layer.workspace)
         if hook is not None:
             hook(layer.counts)
-        moe.moe_popularity_update(layer.counts, layer.hist, layer.step, layer.mean, layer.P,
-                                  layer.hot)
-        layer.step += 1
+        moe.moe_popularity_update_dev(layer.counts, layer.hist, layer.step_dev, layer.mean,
+                                      layer.P, layer.hot)
         ev[2].record(stream)
         moe.moe_dispatch(b["x"], w.k, layer.slot_row, layer.Xp)
         ev[3].record(stream)
@@ -281,17 +286,30 @@ def main():
     for i in range(nb):
         step(i)
         R_of.append(int(layer.offsets[-1].item()))
+    # One CUDA graph per input batch (single rank; multi-rank steps hold an
+    # NCCL call and are issued kernel by kernel).
+    use_graph = world == 1 and not args.no_graph
+    graphs = []
+    if use_graph:
+        for b in batches:
+            graphs.append(layer.capture(b["x"], weights.get("Wg"), weights.get("W1"),
+                                        weights.get("W2"), b["bias"], logits=b.get("logits")))
+
+    def run_step(i):
+        if use_graph:
+            graphs[i % nb].replay()
+        else:
+            step(i)
+
     for i in range(warmup):
-        step(i)
+        run_step(i)
     torch.cuda.synchronize()
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    # ---- timed region (device time, events on the launching stream) ----
-    nev = 6
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(steps)]
+    # ---- timed region: the step as shipped (graph replay), events on the stream ----
     sampler = ClockSampler(local) if rank == 0 else None
     barrier()
     torch.cuda.synchronize()
@@ -301,20 +319,32 @@ def main():
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(steps):
-        step(i, evs[i])
+        run_step(i)
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
-    stage_ms = np.zeros(nev - 1)
-    for e in evs:
-        stage_ms += np.array([e[j].elapsed_time(e[j + 1]) for j in range(nev - 1)])
-    stage_ms /= steps
     if world > 1:
         t = torch.tensor([elapsed_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         elapsed_ms = float(t.item())
+
+    # ---- timed region 2: the same calls issued one by one with an event after
+    # each stage: per-stage device times and the kernels' roofline numbers ----
+    stage_steps = min(steps, 500)
+    nev = 6
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(stage_steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(stage_steps):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    stage_ms = np.zeros(nev - 1)
+    for e in evs:
+        stage_ms += np.array([e[j].elapsed_time(e[j + 1]) for j in range(nev - 1)])
+    stage_ms /= stage_steps
 
     # ---- end to end: pinned host x -> device, layer, y -> pinned host ----
     e2e_steps = max(10, steps // 4)
@@ -329,12 +359,18 @@ def main():
     d2h = host_y.numel() * host_y.element_size()
 
     def e2e_step(i):
-        dx.copy_(host_x[i % nb], non_blocking=True)
-        if dlog is not None:
-            dlog.copy_(host_logits[i % nb], non_blocking=True)
         b = batches[i % nb]
-        layer.forward(dx, weights.get("Wg"), weights.get("W1"), weights.get("W2"), b["bias"],
-                      logits=dlog, counts_hook=hook)
+        if use_graph:  # the graph reads the batch's own device buffers
+            b["x"].copy_(host_x[i % nb], non_blocking=True)
+            if dlog is not None:
+                b["logits"].copy_(host_logits[i % nb], non_blocking=True)
+            graphs[i % nb].replay()
+        else:
+            dx.copy_(host_x[i % nb], non_blocking=True)
+            if dlog is not None:
+                dlog.copy_(host_logits[i % nb], non_blocking=True)
+            layer.forward(dx, weights.get("Wg"), weights.get("W1"), weights.get("W2"), b["bias"],
+                          logits=dlog, counts_hook=hook)
         host_y.copy_(layer.y, non_blocking=True)
 
     for i in range(3):
@@ -357,7 +393,7 @@ def main():
 
     if rank == 0:
         peaks, peak_src = load_peaks()
-        R_mean = float(np.mean([R_of[i % nb] for i in range(steps)]))
+        R_mean = float(np.mean([R_of[i % nb] for i in range(stage_steps)]))
         names = ["gate", "route+popularity", "dispatch", "expert_ffn", "combine"]
         es = 2 if w.dtype == "bf16" else 4
         per = {}
@@ -414,6 +450,10 @@ def main():
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": layer.launches_per_forward(gate=not w.logits_direct) * steps,
                 "roofline": roof, "stages": per, "clocks": clocks, "cpu_baseline": cpu,
+                "timing": {"value": "CUDA-graph replay of the whole step" if use_graph
+                           else "kernels issued one by one (programmatic dependent launch)",
+                           "stages_and_roofline": f"{stage_steps} steps issued stage by stage, "
+                                                  "events between stages"},
                 "device_error_bits": dev_err}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -37,6 +37,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -63,15 +69,15 @@ enum moe_device_error_bits {
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
-const char* moe_status_string(int status);
+MOE_API const char* moe_status_string(int status);
 
 /* Library ABI version: 100 * major + minor. */
-int moe_version(void);
+MOE_API int moe_version(void);
 
 /* Reads the device error word of the CURRENT device (synchronous: waits for
  * all work on the device) into *bits, then clears it if `clear` != 0.
  * Returns MOE_OK or MOE_ERR_CUDA. */
-int moe_device_error(int32_t* bits, int clear);
+MOE_API int moe_device_error(int32_t* bits, int clear);
 
 /* ---------------------------------------------------------------- a0 ----
  * Router logits.  PopFetcher, section 2.1.2: the gate network scores each
@@ -82,7 +88,7 @@ int moe_device_error(int32_t* bits, int clear);
  *                             accumulated in fp32 (bf16 products are exact)
  * T >= 0 (T = 0 launches nothing).  d >= 1.
  */
-int moe_gate(const void* x, const void* Wg, int dtype, int T, int d, int E, float* logits,
+MOE_API int moe_gate(const void* x, const void* Wg, int dtype, int T, int d, int E, float* logits,
              moe_stream_t stream);
 
 /* ---------------------------------------------------------------- a1 ----
@@ -112,9 +118,9 @@ int moe_gate(const void* x, const void* Wg, int dtype, int T, int d, int E, floa
  * Results are bit-identical run to run (no atomics whose order is visible).
  * T = 0 writes zeros to counts, kept, offsets and n_dropped.
  */
-size_t moe_route_workspace_size(int T, int E, int k);
+MOE_API size_t moe_route_workspace_size(int T, int E, int k);
 
-int moe_route(const float* logits, const float* bias, int T, int E, int k, int capacity,
+MOE_API int moe_route(const float* logits, const float* bias, int T, int E, int k, int capacity,
               int32_t* ids, float* w, int32_t* counts, int32_t* kept, int32_t* offsets,
               int32_t* slot_row, int32_t* row_slot, int32_t* n_dropped, void* workspace,
               size_t workspace_bytes, moe_stream_t stream);
@@ -128,7 +134,7 @@ int moe_route(const float* logits, const float* bias, int T, int E, int k, int c
  * 4 MiB device array built into the library (held on every device that loads
  * it until the process exits).
  *  - Size limit: moe_route_workspace_size(T, E, k) <= 4 MiB (e.g. E = 256 up
- *    to T = 262144 tokens, E = 1024 up to T = 65536); larger problems return
+ *    to T = 524032 tokens, E = 1024 up to T = 130816); larger problems return
  *    MOE_ERR_WORKSPACE and launch nothing.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
@@ -138,7 +144,7 @@ int moe_route(const float* logits, const float* bias, int T, int E, int k, int c
  *    the caller.  Nothing in it needs clearing between calls.
  *  - Allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
  */
-int moe_route_noalloc(const float* logits, const float* bias, int T, int E, int k, int capacity,
+MOE_API int moe_route_noalloc(const float* logits, const float* bias, int T, int E, int k, int capacity,
                       int32_t* ids, float* w, int32_t* counts, int32_t* kept, int32_t* offsets,
                       int32_t* slot_row, int32_t* row_slot, int32_t* n_dropped,
                       moe_stream_t stream);
@@ -151,7 +157,7 @@ int moe_route_noalloc(const float* logits, const float* bias, int T, int E, int 
  *   R_max >= R (T*k always suffices).  Rows of Xp that no slot names are left
  *   untouched.  A slot_row entry >= R_max is skipped and flagged on the device.
  */
-int moe_dispatch(const void* x, int dtype, int T, int d, int k, const int32_t* slot_row,
+MOE_API int moe_dispatch(const void* x, int dtype, int T, int d, int k, const int32_t* slot_row,
                  void* Xp, int R_max, moe_stream_t stream);
 
 /* ---------------------------------------------------------------- a3 ----
@@ -168,7 +174,7 @@ int moe_dispatch(const void* x, int dtype, int T, int d, int k, const int32_t* s
  *   Offsets that decrease or exceed R_max are flagged on the device and the
  *   offending expert is skipped.
  */
-int moe_expert_ffn(const void* Xp, const void* W1, const void* W2, int dtype, int E, int d,
+MOE_API int moe_expert_ffn(const void* Xp, const void* W1, const void* W2, int dtype, int E, int d,
                    int F, const int32_t* offsets, int R_max, void* H, void* Yp,
                    moe_stream_t stream);
 
@@ -181,7 +187,7 @@ int moe_expert_ffn(const void* Xp, const void* W1, const void* W2, int dtype, in
  *   whose slots were all dropped gets zeros.
  *   Yp [R_max, d] dtype; slot_row, w [T, k]; y [T, d] dtype.
  */
-int moe_combine(const void* Yp, int dtype, int T, int d, int k, const int32_t* slot_row,
+MOE_API int moe_combine(const void* Yp, int dtype, int T, int d, int k, const int32_t* slot_row,
                 const float* w, void* y, int R_max, moe_stream_t stream);
 
 /* ---------------------------------------------------------------- a5 ----
@@ -199,8 +205,15 @@ int moe_combine(const void* Yp, int dtype, int T, int d, int k, const int32_t* s
  *   The state across steps is hist plus the caller's step counter: copying
  *   hist out and back resumes the sequence exactly.
  */
-int moe_popularity_update(const int32_t* counts, int E, int32_t* hist, int W, int64_t step,
+MOE_API int moe_popularity_update(const int32_t* counts, int E, int32_t* hist, int W, int64_t step,
                           float* mean, int P, int32_t* hot, moe_stream_t stream);
+
+/* The same update with the step counter in device memory: reads *step
+ * (int64, 8-byte aligned device pointer), updates as above, then stores
+ * *step + 1.  A captured CUDA graph that replays the layer therefore advances
+ * the window on every replay.  A negative *step makes the call a no-op. */
+MOE_API int moe_popularity_update_dev(const int32_t* counts, int E, int32_t* hist, int W, int64_t* step,
+                              float* mean, int P, int32_t* hot, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

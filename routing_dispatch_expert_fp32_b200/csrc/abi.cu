@@ -6,10 +6,9 @@ namespace moe {
 __device__ int32_t g_device_error = 0;
 
 int32_t* device_error_word() {
-    constexpr int kMaxDevices = 64;
     static int32_t* cache[kMaxDevices] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    const int dev = current_device();
+    if (dev < 0) return nullptr;
     if (!cache[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
@@ -20,7 +19,7 @@ int32_t* device_error_word() {
 
 }  // namespace moe
 
-extern "C" const char* moe_status_string(int status) {
+extern "C" MOE_API const char* moe_status_string(int status) {
     switch (status) {
         case MOE_OK: return "ok";
         case MOE_ERR_INVALID_ARG: return "invalid argument";
@@ -32,9 +31,9 @@ extern "C" const char* moe_status_string(int status) {
     }
 }
 
-extern "C" int moe_version(void) { return 100; }
+extern "C" MOE_API int moe_version(void) { return 100; }
 
-extern "C" int moe_device_error(int32_t* bits, int clear) {
+extern "C" MOE_API int moe_device_error(int32_t* bits, int clear) {
     if (!bits) return MOE_ERR_INVALID_ARG;
     int32_t v = 0;
     if (cudaMemcpyFromSymbol(&v, moe::g_device_error, sizeof v) != cudaSuccess) return MOE_ERR_CUDA;

@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -33,14 +35,74 @@ inline int launch_status() {
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+constexpr int kMaxDevices = 64;
+
+inline int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+    return dev;
+}
+
+// SM count of the current device (queried once per device).
 inline int num_sms() {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
+    static int cache[kMaxDevices] = {};
+    const int dev = current_device();
+    if (dev < 0) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device (and again only
+// if a larger size is needed), so launches inside a stream capture make no
+// attribute calls.  One static cache per kernel (the kernel is the template
+// argument, so kernels that share a signature do not share a cache).
+template <auto kern>
+inline int ensure_smem(int bytes) {
+    static int done[kMaxDevices] = {};
+    const int dev = current_device();
+    if (dev < 0) return MOE_ERR_CUDA;
+    if (done[dev] >= bytes) return MOE_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    done[dev] = bytes;
+    return MOE_OK;
+}
+
+// Launches `kern` with programmatic stream serialization: the kernel may be
+// scheduled while the previous kernel on the stream is still running, and it
+// waits for that kernel (pdl_wait) before its first global-memory access.
+template <typename... KArgs, typename... Args>
+inline int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // --------------------------------------------------------------- device ----
+// Programmatic dependent launch: wait until the previous kernel on the stream
+// has completed and its writes are visible (returns at once when the kernel
+// was launched without the attribute), and let the next kernel be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // 16-byte global accesses.  Loads of read-only inputs bypass L1 allocation.
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
     uint4 v;

@@ -11,7 +11,7 @@
 
 using namespace moe;
 
-extern "C" int moe_expert_ffn(const void* Xp, const void* W1, const void* W2, int dtype, int E,
+extern "C" MOE_API int moe_expert_ffn(const void* Xp, const void* W1, const void* W2, int dtype, int E,
                               int d, int F, const int32_t* offsets, int R_max, void* H, void* Yp,
                               moe_stream_t stream) {
     if (!dtype_ok(dtype)) return MOE_ERR_UNSUPPORTED;
@@ -37,7 +37,7 @@ extern "C" int moe_expert_ffn(const void* Xp, const void* W1, const void* W2, in
                                 static_cast<float*>(Yp), d, F, E, offsets, 0, R_max, false, st);
 }
 
-extern "C" int moe_gate(const void* x, const void* Wg, int dtype, int T, int d, int E,
+extern "C" MOE_API int moe_gate(const void* x, const void* Wg, int dtype, int T, int d, int E,
                         float* logits, moe_stream_t stream) {
     if (!dtype_ok(dtype)) return MOE_ERR_UNSUPPORTED;
     if (T < 0 || d < 1 || E < 1 || E > kMaxExperts) return MOE_ERR_INVALID_ARG;

@@ -25,12 +25,14 @@ gemm_simt_f32_kernel(const float* __restrict__ A, const float* __restrict__ B,
     __shared__ float As[SBK][SBM + 4];
     __shared__ float Bs[SBK][SBN + 4];
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+    pdl_wait();
+    pdl_trigger();
     const int nt = (N + SBN - 1) / SBN;
     const int total =
-        build_tile_table(offsets, single_M, E, nt, SBM, R_max, s_prefix, s_warp, err);
+        nt * build_tile_table(offsets, single_M, E, 1, SBM, R_max, s_prefix, s_warp, err);
 
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const TileCoord tc = tile_coord(tile, s_prefix, E, offsets, single_M, SBM, SBN);
+        const TileCoord tc = tile_coord(tile, s_prefix, E, offsets, single_M, SBM, SBN, nt);
         const float* Ab = A + (size_t)tc.row0 * K;
         const float* Bb = B + ((size_t)tc.e * N + tc.n0) * K;
         const int ncols = min(SBN, N - tc.n0);
@@ -79,13 +81,8 @@ int launch_gemm_simt_f32(const float* A, const float* B, float* C, int N, int K,
     const int grid = (int)(ub < (long long)num_sms() * 4 ? ub : (long long)num_sms() * 4);
     if (grid <= 0) return MOE_OK;
     int32_t* err = device_error_word();
-    if (relu)
-        gemm_simt_f32_kernel<true><<<grid, SThreads, 0, st>>>(A, B, C, N, K, E, offsets, single_M,
-                                                              R_max, err);
-    else
-        gemm_simt_f32_kernel<false><<<grid, SThreads, 0, st>>>(A, B, C, N, K, E, offsets, single_M,
-                                                               R_max, err);
-    return launch_status();
+    auto kern = relu ? gemm_simt_f32_kernel<true> : gemm_simt_f32_kernel<false>;
+    return launch_pdl(kern, grid, SThreads, 0, st, A, B, C, N, K, E, offsets, single_M, R_max, err);
 }
 
 }  // namespace moe

@@ -76,20 +76,22 @@ __device__ inline int build_tile_table(const int32_t* __restrict__ offsets, int 
     return carry;
 }
 
-// Maps a linear tile index (< s_prefix[E]) to its coordinates.
+// Maps a linear tile index to its coordinates, given the prefix of M-tiles per
+// group (s_prefix from build_tile_table with nt = 1) and nt N-tiles per group:
+// group e owns tiles [nt * s_prefix[e], nt * s_prefix[e+1]).
 __device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* s_prefix, int E,
                                                 const int32_t* __restrict__ offsets, int single_M,
-                                                int BM, int BN) {
-    int lo = 0, hi = E - 1;  // largest e with s_prefix[e] <= tile
+                                                int BM, int BN, int nt) {
+    int lo = 0, hi = E - 1;  // largest e with nt * s_prefix[e] <= tile
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (s_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+        if (nt * s_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
     }
     const int e = lo;
     const int a = group_off(offsets, e, single_M);
     const int m = group_off(offsets, e + 1, single_M) - a;
     const int mt = (m + BM - 1) / BM;
-    const int local = tile - s_prefix[e];
+    const int local = tile - nt * s_prefix[e];
     const int mb = local % mt, nb = local / mt;
     TileCoord c;
     c.e = e;

@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(kPermThreads)
 dispatch_kernel(const uint4* __restrict__ x, int T, int nvec, int k,
                 const int32_t* __restrict__ slot_row, uint4* __restrict__ Xp, int R_max,
                 int32_t* err) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int wpb = kPermThreads / 32;
     const int nwarps = gridDim.x * wpb;
@@ -97,6 +99,8 @@ combine_kernel(const uint4* __restrict__ Yp, int T, int nvec, int k,
                uint4* __restrict__ y, int R_max, int32_t* err) {
     using V = Vec<DT>;
     constexpr int CU = 2;  // vectors per lane per pass (accumulators: CU * V::N floats)
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int wpb = kPermThreads / 32;
     const int nwarps = gridDim.x * wpb;
@@ -162,20 +166,19 @@ static int check_rows(const void* a, const void* b, int dtype, int T, int d, int
 
 using namespace moe;
 
-extern "C" int moe_dispatch(const void* x, int dtype, int T, int d, int k, const int32_t* slot_row,
+extern "C" MOE_API int moe_dispatch(const void* x, int dtype, int T, int d, int k, const int32_t* slot_row,
                             void* Xp, int R_max, moe_stream_t stream) {
     const int rc = check_rows(x, Xp, dtype, T, d, k);
     if (rc != MOE_OK) return rc;
     if (T > 0 && (!slot_row || R_max < 0)) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     const int nvec = (int)((size_t)d * dtype_bytes(dtype) / 16);
-    dispatch_kernel<<<perm_grid(T), kPermThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4*>(x), T, nvec, k, slot_row, static_cast<uint4*>(Xp), R_max,
-        device_error_word());
-    return launch_status();
+    return launch_pdl(dispatch_kernel, perm_grid(T), kPermThreads, 0,
+                      reinterpret_cast<cudaStream_t>(stream), static_cast<const uint4*>(x), T,
+                      nvec, k, slot_row, static_cast<uint4*>(Xp), R_max, device_error_word());
 }
 
-extern "C" int moe_combine(const void* Yp, int dtype, int T, int d, int k, const int32_t* slot_row,
+extern "C" MOE_API int moe_combine(const void* Yp, int dtype, int T, int d, int k, const int32_t* slot_row,
                            const float* w, void* y, int R_max, moe_stream_t stream) {
     const int rc = check_rows(Yp, y, dtype, T, d, k);
     if (rc != MOE_OK) return rc;
@@ -183,13 +186,8 @@ extern "C" int moe_combine(const void* Yp, int dtype, int T, int d, int k, const
     if (T == 0) return MOE_OK;
     const int nvec = (int)((size_t)d * dtype_bytes(dtype) / 16);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (dtype == MOE_DTYPE_BF16)
-        combine_kernel<MOE_DTYPE_BF16><<<perm_grid(T), kPermThreads, 0, st>>>(
-            static_cast<const uint4*>(Yp), T, nvec, k, slot_row, w, static_cast<uint4*>(y), R_max,
-            device_error_word());
-    else
-        combine_kernel<MOE_DTYPE_F32><<<perm_grid(T), kPermThreads, 0, st>>>(
-            static_cast<const uint4*>(Yp), T, nvec, k, slot_row, w, static_cast<uint4*>(y), R_max,
-            device_error_word());
-    return launch_status();
+    auto kern = dtype == MOE_DTYPE_BF16 ? combine_kernel<MOE_DTYPE_BF16>
+                                        : combine_kernel<MOE_DTYPE_F32>;
+    return launch_pdl(kern, perm_grid(T), kPermThreads, 0, st, static_cast<const uint4*>(Yp), T,
+                      nvec, k, slot_row, w, static_cast<uint4*>(y), R_max, device_error_word());
 }

@@ -14,10 +14,17 @@
 
 namespace moe {
 
+// The step comes from `step_ptr` when it is not null (and is advanced by one at
+// the end), else from `step_arg`.
 __global__ void __launch_bounds__(1024)
 popularity_kernel(const int32_t* __restrict__ counts, int E, int32_t* __restrict__ hist, int W,
-                  long long step, float* __restrict__ mean, int P, int32_t* __restrict__ hot) {
+                  long long step_arg, long long* step_ptr, float* __restrict__ mean, int P,
+                  int32_t* __restrict__ hot) {
     __shared__ long long s_sum[kMaxExperts];
+    pdl_wait();
+    pdl_trigger();
+    const long long step = step_ptr ? *step_ptr : step_arg;
+    if (step < 0) return;
     const int slot = (int)(step % W);
     const long long n = step + 1 < W ? step + 1 : W;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -41,18 +48,33 @@ popularity_kernel(const int32_t* __restrict__ counts, int E, int32_t* __restrict
         }
         if (rank < P) hot[rank] = e;
     }
+    if (step_ptr) {
+        __syncthreads();  // every thread has read the step
+        if (threadIdx.x == 0) *step_ptr = step + 1;
+    }
 }
 
 }  // namespace moe
 
-extern "C" int moe_popularity_update(const int32_t* counts, int E, int32_t* hist, int W,
+extern "C" MOE_API int moe_popularity_update(const int32_t* counts, int E, int32_t* hist, int W,
                                      int64_t step, float* mean, int P, int32_t* hot,
                                      moe_stream_t stream) {
     using namespace moe;
     if (E < 1 || E > kMaxExperts || W < 1 || step < 0 || P < 0 || P > E) return MOE_ERR_INVALID_ARG;
     if (!counts || !hist || !mean || (P > 0 && !hot)) return MOE_ERR_INVALID_ARG;
     const int threads = ((E + 31) / 32) * 32;
-    popularity_kernel<<<1, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        counts, E, hist, W, (long long)step, mean, P, hot);
-    return launch_status();
+    return launch_pdl(popularity_kernel, 1, threads, 0, reinterpret_cast<cudaStream_t>(stream),
+                      counts, E, hist, W, (long long)step, (long long*)nullptr, mean, P, hot);
+}
+
+extern "C" MOE_API int moe_popularity_update_dev(const int32_t* counts, int E, int32_t* hist, int W,
+                                         int64_t* step, float* mean, int P, int32_t* hot,
+                                         moe_stream_t stream) {
+    using namespace moe;
+    if (E < 1 || E > kMaxExperts || W < 1 || P < 0 || P > E) return MOE_ERR_INVALID_ARG;
+    if (!counts || !hist || !mean || !step || (P > 0 && !hot)) return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(step) & 7u) != 0) return MOE_ERR_UNSUPPORTED;
+    const int threads = ((E + 31) / 32) * 32;
+    return launch_pdl(popularity_kernel, 1, threads, 0, reinterpret_cast<cudaStream_t>(stream),
+                      counts, E, hist, W, 0LL, reinterpret_cast<long long*>(step), mean, P, hot);
 }

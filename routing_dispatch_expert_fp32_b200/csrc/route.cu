@@ -4,7 +4,9 @@
 // under an expert-capacity limit) and PopFetcher, section 2.1.2 (top-k gate).
 //
 // Three launches, no inter-CTA waiting:
-//   K1 route_topk    one CTA per chunk of 128 tokens.  A group of L lanes
+//   K1 route_topk    one CTA of 32 warps (8 for E > 256) per chunk of 256 tokens (8 per warp;
+//                    the next token's logits are loaded while the current one
+//                    is ranked).  A group of L lanes
 //                    (L = 8, 16 or 32) scores one token: each lane holds E/L
 //                    of the fp32 keys z = logit + bias (coalesced loads), k
 //                    rounds of a butterfly argmax under the total order
@@ -16,7 +18,7 @@
 //                    histograms (two-level: segments of chunks, then chunks),
 //                    counts, kept = min(counts, capacity), offsets = exclusive
 //                    scan of kept, n_dropped.
-//   K3 route_assign  one CTA per chunk again; a slot's position inside its
+//   K3 route_assign  one CTA per chunk again (a token per thread); a slot's position inside its
 //                    expert = chunk base + slots of earlier warps of the chunk
 //                    + earlier lanes of its warp, all from per-warp lane masks
 //                    (atomicOr commutes; popc of the lower-lane bits gives the
@@ -27,8 +29,12 @@
 
 namespace moe {
 
-constexpr int kChunk = 128;   // tokens per chunk (= per CTA in K1 and K3)
-constexpr int kThreads = 128; // 4 warps, 32 tokens each
+constexpr int kChunk = 256;        // tokens per chunk (= per CTA in K1 and K3)
+// K1 threads: 32 warps (kChunk / 32 tokens each); 8 warps when a lane holds
+// 16 or more keys, so the keys of two tokens stay in registers.
+template <int VPL>
+constexpr int topk_threads() { return VPL >= 16 ? 256 : 1024; }
+constexpr int kThreads = kChunk;   // K3: one token per thread
 constexpr int kWarps = kThreads / 32;
 constexpr int kScanThreads = 1024;
 
@@ -38,15 +44,20 @@ __device__ __forceinline__ bool key_better(float av, int ai, float bv, int bi) {
 
 // ------------------------------------------------------------------- K1 ----
 template <int L, int VPL>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(topk_threads<VPL>())
 route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
                   int k, int32_t* __restrict__ ids, float* __restrict__ w,
                   int32_t* __restrict__ chunk_hist) {
     __shared__ int s_hist[kMaxExperts];
-    for (int e = threadIdx.x; e < E; e += kThreads) s_hist[e] = 0;
+    constexpr int kTopkThreads = topk_threads<VPL>();
+    for (int e = threadIdx.x; e < E; e += kTopkThreads) s_hist[e] = 0;
     __syncthreads();
+    pdl_wait();
+    pdl_trigger();
 
-    constexpr int G = 32 / L;  // tokens per warp per iteration
+    constexpr int G = 32 / L;                          // tokens per warp per iteration
+    constexpr int kPerWarp = kChunk / (kTopkThreads / 32);
+    constexpr int kIters = kPerWarp / G;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane / L, gl = lane % L;
 
@@ -58,17 +69,33 @@ route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bi
         b[i] = (bias != nullptr && e < E) ? bias[e] : 0.0f;
     }
 
-    const int t_warp = blockIdx.x * kChunk + warp * 32;
-    for (int it = 0; it < 32 / G; ++it) {
+    const int t_warp = blockIdx.x * kChunk + warp * kPerWarp;
+    float zn[VPL];  // logits of the next token of this group, in flight
+    {
+        const int t = min(t_warp + g, T - 1);
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int e = gl + i * L;
+            zn[i] = (e < E) ? __ldg(logits + (size_t)t * E + e) : 0.0f;
+        }
+    }
+#pragma unroll 1
+    for (int it = 0; it < kIters; ++it) {
         const int t = t_warp + it * G + g;
         const bool active = t < T;
-        const float* row = logits + (size_t)(active ? t : T - 1) * E;
-
         float z[VPL];
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
             const int e = gl + i * L;
-            z[i] = (e < E) ? __fadd_rn(__ldg(row + e), b[i]) : -INFINITY;
+            z[i] = (e < E) ? __fadd_rn(zn[i], b[i]) : -INFINITY;
+        }
+        if (it + 1 < kIters) {
+            const int tn = min(t + G, T - 1);
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int e = gl + i * L;
+                zn[i] = (e < E) ? __ldg(logits + (size_t)tn * E + e) : 0.0f;
+            }
         }
 
         uint32_t taken = 0;
@@ -113,7 +140,7 @@ route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bi
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += kThreads)
+    for (int e = threadIdx.x; e < E; e += kTopkThreads)
         chunk_hist[(size_t)blockIdx.x * E + e] = s_hist[e];
 }
 
@@ -125,6 +152,8 @@ route_scan_kernel(const int32_t* __restrict__ chunk_hist, int nchunks, int T, in
                   int32_t* __restrict__ n_dropped) {
     __shared__ int32_t s_seg[kScanThreads];  // [segment][expert]
     __shared__ int32_t s_warp[kScanThreads / 32];
+    pdl_wait();
+    pdl_trigger();
     const int tid = threadIdx.x;
     const int S = kScanThreads / E;              // segments (E <= 1024 so S >= 1)
     const int cps = (nchunks + S - 1) / S;       // chunks per segment
@@ -134,8 +163,10 @@ route_scan_kernel(const int32_t* __restrict__ chunk_hist, int nchunks, int T, in
 
     // phase 1: per (segment, expert) totals
     int32_t part = 0;
-    if (worker)
+    if (worker) {
+#pragma unroll 8
         for (int c = c0; c < c1; ++c) part += chunk_hist[(size_t)c * E + e];
+    }
     if (worker) s_seg[seg * E + e] = part;
     __syncthreads();
 
@@ -157,6 +188,7 @@ route_scan_kernel(const int32_t* __restrict__ chunk_hist, int nchunks, int T, in
     // phase 3: per chunk bases
     if (worker) {
         int32_t run = s_seg[seg * E + e];
+#pragma unroll 8
         for (int c = c0; c < c1; ++c) {
             const int32_t v = chunk_hist[(size_t)c * E + e];
             chunk_base[(size_t)c * E + e] = run;
@@ -201,6 +233,8 @@ route_assign_kernel(const int32_t* __restrict__ ids, int T, int E, int k, int ca
     __shared__ uint32_t s_mask[kWarps][kMaxExperts];
     __shared__ int32_t s_base[kMaxExperts];
     __shared__ int32_t s_off[kMaxExperts];
+    pdl_wait();
+    pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int e = tid; e < E; e += kThreads) {
         s_base[e] = chunk_base[(size_t)blockIdx.x * E + e];
@@ -238,61 +272,84 @@ route_assign_kernel(const int32_t* __restrict__ ids, int T, int E, int k, int ca
 static size_t align256(size_t v) { return (v + 255u) & ~size_t(255u); }
 
 template <int L, int VPL>
-static void launch_topk(int nchunks, cudaStream_t st, const float* logits, const float* bias,
-                        int T, int E, int k, int32_t* ids, float* w, int32_t* hist) {
-    route_topk_kernel<L, VPL><<<nchunks, kThreads, 0, st>>>(logits, bias, T, E, k, ids, w, hist);
+static int launch_topk(int nchunks, cudaStream_t st, const float* logits, const float* bias,
+                       int T, int E, int k, int32_t* ids, float* w, int32_t* hist) {
+    return launch_pdl(route_topk_kernel<L, VPL>, nchunks, topk_threads<VPL>(), 0, st, logits, bias,
+                      T, E, k, ids, w, hist);
+}
+
+// The three launches of one routing call; `scratch` is 256-byte aligned and
+// holds at least route_scratch_bytes(T, E).
+static size_t route_scratch_bytes(int T, int E) {
+    const size_t nchunks = ((size_t)T + kChunk - 1) / kChunk;
+    return 2 * align256(nchunks * (size_t)E * sizeof(int32_t));
+}
+
+static int launch_route(const float* logits, const float* bias, int T, int E, int k, int capacity,
+                        int32_t* ids, float* w, int32_t* counts, int32_t* kept, int32_t* offsets,
+                        int32_t* slot_row, int32_t* row_slot, int32_t* n_dropped, char* scratch,
+                        cudaStream_t st) {
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    int32_t* hist = reinterpret_cast<int32_t*>(scratch);
+    int32_t* base = reinterpret_cast<int32_t*>(scratch + align256((size_t)nchunks * E * 4));
+    if (T > 0) {
+        int rc;
+        if (E <= 8) rc = launch_topk<8, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 16) rc = launch_topk<16, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 32) rc = launch_topk<32, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 64) rc = launch_topk<32, 2>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 128) rc = launch_topk<32, 4>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 256) rc = launch_topk<32, 8>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else if (E <= 512) rc = launch_topk<32, 16>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        else rc = launch_topk<32, 32>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        if (rc != MOE_OK) return MOE_ERR_CUDA;
+    }
+    if (launch_pdl(route_scan_kernel, 1, kScanThreads, 0, st, (const int32_t*)hist, nchunks, T, E,
+                   k, capacity, base, counts, kept, offsets, n_dropped) != MOE_OK)
+        return MOE_ERR_CUDA;
+    if (T > 0) {
+        if (launch_pdl(route_assign_kernel, nchunks, kThreads, 0, st, (const int32_t*)ids, T, E, k,
+                       capacity, (const int32_t*)base, (const int32_t*)offsets, slot_row,
+                       row_slot) != MOE_OK)
+            return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+static int check_route_args(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                            int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* slot_row,
+                            int32_t* row_slot, int32_t* n_dropped) {
+    if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > kMaxTopK)
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)T * k >= INT32_MAX) return MOE_ERR_INVALID_ARG;
+    if (!counts || !kept || !offsets || !n_dropped) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !ids || !w || !slot_row || !row_slot)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
 }
 
 }  // namespace moe
 
 using namespace moe;
 
-extern "C" size_t moe_route_workspace_size(int T, int E, int k) {
+extern "C" MOE_API size_t moe_route_workspace_size(int T, int E, int k) {
     (void)k;
     if (T < 0 || E <= 0) return 0;
-    const size_t nchunks = ((size_t)T + kChunk - 1) / kChunk;
-    return 2 * align256(nchunks * (size_t)E * sizeof(int32_t)) + 256;
+    return route_scratch_bytes(T, E) + 256;  // + slack to align the caller's pointer
 }
 
-extern "C" int moe_route(const float* logits, const float* bias, int T, int E, int k, int capacity,
+extern "C" MOE_API int moe_route(const float* logits, const float* bias, int T, int E, int k, int capacity,
                          int32_t* ids, float* w, int32_t* counts, int32_t* kept, int32_t* offsets,
                          int32_t* slot_row, int32_t* row_slot, int32_t* n_dropped, void* workspace,
                          size_t workspace_bytes, moe_stream_t stream) {
-    if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > kMaxTopK)
-        return MOE_ERR_INVALID_ARG;
-    if ((int64_t)T * k >= INT32_MAX) return MOE_ERR_INVALID_ARG;
-    if (!counts || !kept || !offsets || !n_dropped) return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (!logits || !ids || !w || !slot_row || !row_slot)) return MOE_ERR_INVALID_ARG;
+    const int rc = check_route_args(logits, T, E, k, ids, w, counts, kept, offsets, slot_row,
+                                    row_slot, n_dropped);
+    if (rc != MOE_OK) return rc;
     const size_t need = moe_route_workspace_size(T, E, k);
     if (!workspace || workspace_bytes < need) return MOE_ERR_WORKSPACE;
-
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int nchunks = (T + kChunk - 1) / kChunk;
     char* ws = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(workspace) + 255u) &
                                        ~uintptr_t(255u));
-    int32_t* hist = reinterpret_cast<int32_t*>(ws);
-    int32_t* base = reinterpret_cast<int32_t*>(ws + align256((size_t)nchunks * E * 4));
-
-    if (T > 0) {
-        if (E <= 8) launch_topk<8, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 16) launch_topk<16, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 32) launch_topk<32, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 64) launch_topk<32, 2>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 128) launch_topk<32, 4>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 256) launch_topk<32, 8>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 512) launch_topk<32, 16>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else launch_topk<32, 32>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
-    }
-    route_scan_kernel<<<1, kScanThreads, 0, st>>>(hist, nchunks, T, E, k, capacity, base, counts,
-                                                  kept, offsets, n_dropped);
-    if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
-    if (T > 0) {
-        route_assign_kernel<<<nchunks, kThreads, 0, st>>>(ids, T, E, k, capacity, base, offsets,
-                                                          slot_row, row_slot);
-        if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
-    }
-    return MOE_OK;
+    return launch_route(logits, bias, T, E, k, capacity, ids, w, counts, kept, offsets, slot_row,
+                        row_slot, n_dropped, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------------------
@@ -333,44 +390,18 @@ static void* noalloc_scratch_ptr() {
 
 }  // namespace moe
 
-extern "C" int moe_route_noalloc(const float* logits, const float* bias, int T, int E, int k,
+extern "C" MOE_API int moe_route_noalloc(const float* logits, const float* bias, int T, int E, int k,
                                  int capacity, int32_t* ids, float* w, int32_t* counts,
                                  int32_t* kept, int32_t* offsets, int32_t* slot_row,
                                  int32_t* row_slot, int32_t* n_dropped, moe_stream_t stream) {
-    if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > kMaxTopK)
-        return MOE_ERR_INVALID_ARG;
-    if ((int64_t)T * k >= INT32_MAX) return MOE_ERR_INVALID_ARG;
-    if (!counts || !kept || !offsets || !n_dropped) return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (!logits || !ids || !w || !slot_row || !row_slot)) return MOE_ERR_INVALID_ARG;
+    const int rc = check_route_args(logits, T, E, k, ids, w, counts, kept, offsets, slot_row,
+                                    row_slot, n_dropped);
+    if (rc != MOE_OK) return rc;
     // The fixed scratch bounds the problem size.
     if (moe_route_workspace_size(T, E, k) > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
     void* scratch = noalloc_scratch_ptr();
     if (!scratch) return MOE_ERR_CUDA;
-
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int nchunks = (T + kChunk - 1) / kChunk;
-    char* ws = static_cast<char*>(scratch);  // 256-byte aligned by declaration
-    int32_t* hist = reinterpret_cast<int32_t*>(ws);
-    int32_t* base = reinterpret_cast<int32_t*>(ws + align256((size_t)nchunks * E * 4));
-
-    if (T > 0) {
-        if (E <= 8) launch_topk<8, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 16) launch_topk<16, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 32) launch_topk<32, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 64) launch_topk<32, 2>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 128) launch_topk<32, 4>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 256) launch_topk<32, 8>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 512) launch_topk<32, 16>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else launch_topk<32, 32>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
-    }
-    route_scan_kernel<<<1, kScanThreads, 0, st>>>(hist, nchunks, T, E, k, capacity, base, counts,
-                                                  kept, offsets, n_dropped);
-    if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
-    if (T > 0) {
-        route_assign_kernel<<<nchunks, kThreads, 0, st>>>(ids, T, E, k, capacity, base, offsets,
-                                                          slot_row, row_slot);
-        if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
-    }
-    return MOE_OK;
+    return launch_route(logits, bias, T, E, k, capacity, ids, w, counts, kept, offsets, slot_row,
+                        row_slot, n_dropped, static_cast<char*>(scratch),
+                        reinterpret_cast<cudaStream_t>(stream));
 }

@@ -38,6 +38,8 @@ _SIGS = {
     "moe_expert_ffn": ([_p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _p, _p], _i),
     "moe_combine": ([_p, _i, _i, _i, _i, _p, _p, _p, _i, _p], _i),
     "moe_popularity_update": ([_p, _i, _p, _i, _i64, _p, _i, _p, _p], _i),
+    "moe_popularity_update_dev": ([_p, _i, _p, _i, _p, _p, _i, _p, _p], _i),
+    "moe_route_noalloc": ([_p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -128,12 +130,31 @@ def moe_popularity_update(counts, hist, step, mean, P, hot, stream=None):
         _ptr(counts), E, _ptr(hist), W, int(step), _ptr(mean), P, _ptr(hot), _stream(stream)))
 
 
+def moe_popularity_update_dev(counts, hist, step_dev, mean, P, hot, stream=None):
+    """step_dev: int64 device tensor of one element, advanced by the call."""
+    W, E = hist.shape
+    _check("moe_popularity_update_dev", lib.moe_popularity_update_dev(
+        _ptr(counts), E, _ptr(hist), W, _ptr(step_dev), _ptr(mean), P, _ptr(hot),
+        _stream(stream)))
+
+
+def moe_route_noalloc(logits, bias, k, capacity, ids, w, counts, kept, offsets, slot_row,
+                      row_slot, n_dropped, stream=None):
+    T, E = logits.shape
+    _check("moe_route_noalloc", lib.moe_route_noalloc(
+        _ptr(logits), _ptr(bias), T, E, k, int(capacity), _ptr(ids), _ptr(w), _ptr(counts),
+        _ptr(kept), _ptr(offsets), _ptr(slot_row), _ptr(row_slot), _ptr(n_dropped),
+        _stream(stream)))
+
+
 class MoELayer:
     """One MoE layer's device buffers plus the call sequence of the hot path.
 
     Weights stay resident; ``forward`` runs gate (unless logits are given),
     route, popularity, dispatch, expert FFN and combine on the current stream,
     all through the C ABI.  ``identity_experts`` skips the FFN (Yp = Xp).
+    The popularity step counter lives in device memory (``step_dev``), so a
+    forward captured by ``capture`` keeps advancing the window on replay.
     """
 
     def __init__(self, T, d, E, k, F, dtype, capacity=0, W=4, P=8, device="cuda",
@@ -161,7 +182,7 @@ class MoELayer:
         self.hist = torch.zeros(W, E, dtype=i32, device=dev)
         self.mean = torch.empty(E, dtype=torch.float32, device=dev)
         self.hot = torch.empty(max(P, 1), dtype=i32, device=dev)
-        self.step = 0
+        self.step_dev = torch.zeros(1, dtype=torch.int64, device=dev)
 
     def forward(self, x, Wg=None, W1=None, W2=None, bias=None, logits=None, stream=None,
                 popularity=True, counts_hook=None):
@@ -174,14 +195,30 @@ class MoELayer:
         if popularity:
             if counts_hook is not None:  # e.g. an all_reduce of the counts across ranks
                 counts_hook(self.counts)
-            moe_popularity_update(self.counts, self.hist, self.step, self.mean, self.P, self.hot,
-                                  stream)
-            self.step += 1
+            moe_popularity_update_dev(self.counts, self.hist, self.step_dev, self.mean, self.P,
+                                      self.hot, stream)
         moe_dispatch(x, self.k, self.slot_row, self.Xp, stream)
         if not self.identity_experts:
             moe_expert_ffn(self.Xp, W1, W2, self.offsets, self.H, self.Yp, stream)
         moe_combine(self.Yp, self.k, self.slot_row, self.w, self.y, stream)
         return self.y
+
+    def capture(self, x, Wg=None, W1=None, W2=None, bias=None, logits=None, popularity=True):
+        """Records one ``forward`` on these tensors into a CUDA graph and returns it.
+
+        ``graph.replay()`` then reruns the whole layer on whatever the captured
+        tensors hold (copy new tokens into ``x`` first).  Capturing runs the
+        layer once (torch's warm-up), which advances the popularity window.
+        """
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.forward(x, Wg, W1, W2, bias, logits=logits, popularity=popularity)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.forward(x, Wg, W1, W2, bias, logits=logits, popularity=popularity)
+        return graph
 
     def launches_per_forward(self, gate=True, popularity=True) -> int:
         """Kernel launches one forward makes (route is three kernels)."""

@@ -147,3 +147,28 @@ def test_layer_bw_sweep_identity_experts(moe, T, s):
     w = wl.WORKLOADS["bw_sweep"].with_(T=T, zipf_s=s)
     layer = make_layer(moe, w)
     check_layer(moe, w, wl.make_step(w, 0), {}, layer, np.random.default_rng(3))
+
+
+def test_graph_replay_matches_eager_and_advances_the_window(moe):
+    w = wl.tiny("graph", T=700, d=256, E=12, k=2, F=384, zipf_s=1.1, W=3, P=4)
+    weights = {k: dev(v) for k, v in wl.make_weights(w).items()}
+    steps = [wl.make_step(w, s) for s in range(5)]
+    x = dev(steps[0]["x"]).clone()
+    bias = dev(steps[0]["bias"]).clone()
+    graphed, eager = make_layer(moe, w), make_layer(moe, w)
+    g = graphed.capture(x, weights["Wg"], weights["W1"], weights["W2"], bias)
+    graphed.hist.zero_()
+    graphed.step_dev.zero_()  # the capture's warm-up forward advanced the window
+    hist_ref = np.zeros((w.W, w.E), np.int32)
+    for s, inp in enumerate(steps):
+        x.copy_(dev(inp["x"]))
+        g.replay()
+        y_e = eager.forward(dev(inp["x"]), weights["Wg"], weights["W1"], weights["W2"], bias)
+        torch.cuda.synchronize()
+        assert torch.equal(graphed.y, y_e), s
+        r = oracle.route(host(graphed.logits), host(bias), w.k, w.capacity)
+        mean_ref, hot_ref = oracle.popularity_update(r["counts"], hist_ref, s, w.P)
+        assert np.array_equal(host(graphed.mean), mean_ref), s
+        assert np.array_equal(host(graphed.hot)[: w.P], hot_ref), s
+    assert int(graphed.step_dev.item()) == len(steps)
+    assert moe.moe_device_error() == 0
