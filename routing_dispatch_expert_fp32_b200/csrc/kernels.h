@@ -17,4 +17,10 @@ int launch_gemm_tc_bf16(const void* A, const void* B, void* C, bool out_f32, int
                         const int32_t* offsets, int single_M, int R_max, bool relu,
                         cudaStream_t st);
 
+// Router logits for E <= 32 on the CUDA cores (gate.cu); gate_small_fits says
+// whether the gate weights fit the kernel's shared-memory stage.
+bool gate_small_fits(int E, int d, int dtype);
+int launch_gate_small(const void* x, const void* Wg, int dtype, int T, int d, int E,
+                      float* logits, cudaStream_t st);
+
 }  // namespace moe

@@ -42,6 +42,16 @@ __device__ __forceinline__ bool key_better(float av, int ai, float bv, int bi) {
     return av > bv || (av == bv && ai < bi);
 }
 
+// Order-preserving map of a finite fp32 to uint32 (larger float -> larger
+// key); -0.0 is folded onto +0.0 first so that the two still tie.
+__device__ __forceinline__ uint32_t order_key(float z) {
+    const uint32_t u = __float_as_uint(z == 0.0f ? 0.0f : z);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // ------------------------------------------------------------------- K1 ----
 template <int L, int VPL>
 __global__ void __launch_bounds__(topk_threads<VPL>())
@@ -101,31 +111,58 @@ route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bi
         uint32_t taken = 0;
         float my_z = 0.0f;
         int my_e = 0;
-        for (int r = 0; r < k; ++r) {
-            float bv = -INFINITY;
-            int bi = INT_MAX;
+        if constexpr (L == 32) {
+            // One token per warp: per round, the largest order key by a warp
+            // reduction, then the lowest expert index among the lanes holding
+            // it (each lane's candidate is its own lowest-index maximum).
+            uint32_t key[VPL];
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int e = gl + i * L;
-                if (e < E && !((taken >> i) & 1u) && key_better(z[i], e, bv, bi)) {
-                    bv = z[i];
-                    bi = e;
+            for (int i = 0; i < VPL; ++i) key[i] = (gl + i * L < E) ? order_key(z[i]) : 0u;
+            for (int r = 0; r < k; ++r) {
+                uint32_t bk = 0u;
+                int bi = INT_MAX;
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    if (!((taken >> i) & 1u) && key[i] > bk) {
+                        bk = key[i];
+                        bi = gl + i * L;
+                    }
+                }
+                const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+                const int win = (int)__reduce_min_sync(0xffffffffu, bk == m ? (uint32_t)bi : 0xffffffffu);
+                if (win % L == gl) taken |= 1u << (win / L);
+                if (gl == r) {
+                    my_z = key_value(m);
+                    my_e = win;
                 }
             }
+        } else {
+            for (int r = 0; r < k; ++r) {
+                float bv = -INFINITY;
+                int bi = INT_MAX;
 #pragma unroll
-            for (int off = L / 2; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off, L);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, off, L);
-                if (key_better(ov, oi, bv, bi)) {
-                    bv = ov;
-                    bi = oi;
+                for (int i = 0; i < VPL; ++i) {
+                    const int e = gl + i * L;
+                    if (e < E && !((taken >> i) & 1u) && key_better(z[i], e, bv, bi)) {
+                        bv = z[i];
+                        bi = e;
+                    }
                 }
-            }
-            // every lane of the group now holds the same winner
-            if (bi % L == gl) taken |= 1u << (bi / L);
-            if (gl == r) {
-                my_z = bv;
-                my_e = bi;
+#pragma unroll
+                for (int off = L / 2; off > 0; off >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off, L);
+                    const int oi = __shfl_xor_sync(0xffffffffu, bi, off, L);
+                    if (key_better(ov, oi, bv, bi)) {
+                        bv = ov;
+                        bi = oi;
+                    }
+                }
+                // every lane of the group now holds the same winner
+                if (bi % L == gl) taken |= 1u << (bi / L);
+                if (gl == r) {
+                    my_z = bv;
+                    my_e = bi;
+                }
             }
         }
 

@@ -87,9 +87,12 @@ def test_ffn_bad_offsets_are_flagged_not_followed(moe):
     assert moe.moe_device_error() & moe.MOE_DEVERR_OFFSETS
 
 
-@pytest.mark.parametrize("T,d,E,dtype", [(512, 64, 8, "f32"), (4096, 1024, 16, "bf16"),
-                                         (1000, 136, 300, "bf16"), (333, 200, 6, "bf16"),
-                                         (16384, 2048, 64, "bf16"), (130, 64, 20, "f32")])
+@pytest.mark.parametrize("T,d,E,dtype", [
+    (512, 64, 8, "f32"), (4096, 1024, 16, "bf16"),        # CUDA-core gate (E <= 32)
+    (333, 200, 6, "bf16"), (130, 64, 20, "f32"), (1001, 1024, 32, "bf16"), (7, 512, 1, "bf16"),
+    (1000, 136, 300, "bf16"), (16384, 2048, 64, "bf16"),  # tensor-core gate
+    (200, 4096, 32, "bf16"),                              # E <= 32 but Wg too big to stage
+])
 def test_gate_matches_oracle(moe, T, d, E, dtype):
     x = rand((T, d), 1.0, dtype, 5)
     Wg = rand((E, d), d ** -0.5, dtype, 6)
