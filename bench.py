@@ -82,6 +82,31 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+GEMM_SOURCES = ["gemm_tc.cu", "grouped.cuh", "common.cuh"]
+
+
+def gemm_traffic(workload: str):
+    """Measured DRAM bytes per launch of the grouped GEMM from profiles/traffic.md,
+    or None when missing or taken on different kernel sources."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "routing_dispatch_expert_fp32_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    sha = h.hexdigest()[:16]
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) == 4 and cells[0] == workload and cells[3] == sha:
+            try:
+                return int(cells[2])
+            except ValueError:
+                return None
+    return None
+
+
 def config_of(w: wl.Workload, n: int):
     c = {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "F": w.F,
          "capacity": w.capacity, "zipf_s": w.zipf_s, "global_batch_tokens": w.T * n,
@@ -433,7 +458,9 @@ def main():
                 roof["kernel"] = "gemm_simt_f32_kernel"
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["peak_source"] = f"{peak_src} ({'bf16_tflops_sustained' if roof['unit'] == 'TFLOP/s' else 'hbm_gbs'})"
-        roof["traffic"] = None
+        roof["traffic"] = (gemm_traffic(w.name)
+                           if roof["kernel"] == "gemm_tc_kernel" and args.tokens == 0
+                           and args.experts == 0 else None)
         value = w.T * steps * world / (elapsed_ms * 1e-3)
         cpu = None
         if world == 1 and args.cpu_seconds > 0:

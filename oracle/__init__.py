@@ -70,6 +70,10 @@ def _load():
         lib.oracle_combine.restype = None
         lib.oracle_popularity_update.argtypes = [p, i32, p, i32, i64, p, i32, p]
         lib.oracle_popularity_update.restype = i32
+        lib.oracle_correlation_update.argtypes = [p, i32, p, i32, i32, i32, p]
+        lib.oracle_correlation_update.restype = None
+        lib.oracle_popularity_forecast.argtypes = [p, p, i32, i32, i32, p, i32, p]
+        lib.oracle_popularity_forecast.restype = None
         lib.oracle_round_bf16.argtypes = [ctypes.c_double]
         lib.oracle_round_bf16.restype = ctypes.c_uint16
         _lib = lib
@@ -207,6 +211,27 @@ def popularity_update(counts: np.ndarray, hist: np.ndarray, step: int, P: int):
     if rc != 0:
         raise ValueError("oracle_popularity_update: invalid sizes")
     return mean, hot[:P].copy()
+
+
+def correlation_update(ids_prev: np.ndarray, ids_next: np.ndarray, C: np.ndarray) -> None:
+    """Adds the consecutive-layer co-selection counts of one batch into C [E,E] (in place)."""
+    a, b = _c(ids_prev, np.int32), _c(ids_next, np.int32)
+    assert C.dtype == np.int32 and C.flags.c_contiguous and a.shape[0] == b.shape[0]
+    T = a.shape[0]
+    _load().oracle_correlation_update(_ptr(a), a.shape[1], _ptr(b), b.shape[1], T, C.shape[0],
+                                      _ptr(C))
+
+
+def popularity_forecast(pop_prev: np.ndarray, C: np.ndarray, k_prev: int, k_next: int, P: int):
+    """Next-layer popularity forecast (fp32 [E]) and its top-P experts."""
+    pop = _c(pop_prev, np.float32)
+    Cc = _c(C, np.int32)
+    E = Cc.shape[0]
+    pred = np.empty(E, np.float32)
+    hot = np.empty(max(P, 1), np.int32)
+    _load().oracle_popularity_forecast(_ptr(pop), _ptr(Cc), E, k_prev, k_next, _ptr(pred), P,
+                                       _ptr(hot))
+    return pred, hot[:P].copy()
 
 
 def layer(x, Wg, W1, W2, bias, k, capacity=0, logits=None):

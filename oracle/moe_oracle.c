@@ -27,6 +27,12 @@
  *               distribution of recent iterations over a sliding window of s
  *               iterations.  Reading taken: the arithmetic mean of the last
  *               n = min(steps seen, W) per-expert count vectors.
+ *   [Pop-4.1]   PopFetcher, section 4.1 (Fig. 6): a token's expert choices at two
+ *               consecutive layers form a correlated pair; the next layer's hot
+ *               experts follow from the previous layer's choices.
+ *   [Pop-4.2b]  PopFetcher, section 4.2, Eq. 2-3 (lost): the conditional
+ *               probability of the next-layer expert given the previous-layer
+ *               one, and the correlation-based popularity forecast.
  *   [MPMC]      MoE-MPMC summary, problem statement item 3: routing is softmax
  *               based.
  *
@@ -325,4 +331,63 @@ int oracle_popularity_update(const int32_t* counts, int E, int32_t* hist, int W,
     free(sum);
     free(taken);
     return 0;
+}
+
+/* ------------------------------------------- cross-layer correlation (f2) -- */
+
+/* Co-selection counts between consecutive MoE layers.  PopFetcher, section 4.1
+ * (Fig. 6): a token that picks expert x at layer j and x' at layer j+1 forms a
+ * correlated pair (x, x').  Every token t adds one to C[i][h] for each i among
+ * its layer-j experts and each h among its layer-(j+1) experts.  C is [E][E]
+ * int32 and is accumulated into (not cleared). */
+void oracle_correlation_update(const int32_t* ids_prev, int k_prev, const int32_t* ids_next,
+                               int k_next, int T, int E, int32_t* C) {
+    for (int t = 0; t < T; ++t)
+        for (int a = 0; a < k_prev; ++a)
+            for (int b = 0; b < k_next; ++b) {
+                int i = ids_prev[(int64_t)t * k_prev + a];
+                int h = ids_next[(int64_t)t * k_next + b];
+                C[(int64_t)i * E + h] += 1;
+            }
+}
+
+/* Correlation-based popularity forecast.  PopFetcher, section 4.2, Eq. 2-3
+ * (lost in extraction): the conditional probability that a token which chose
+ * expert i at layer j chooses h at layer j+1, and the next layer's popularity
+ * predicted from the previous layer's.  Reading taken:
+ *   n_i     = tokens that chose i at layer j = (sum_h C[i][h]) / k_next
+ *   P(h|i)  = C[i][h] / n_i                     (sum_h P(h|i) = k_next)
+ *   pred[h] = sum_i pop_prev[i] * P(h|i) / k_prev
+ * (pop_prev counts token-slots, each token k_prev times; rows with n_i = 0 add
+ * nothing).  Evaluated in double in this fixed order, then rounded once to
+ * fp32:  S_i = sum_h C[i][h];  q_i = (pop_prev[i] * k_next) / (S_i * k_prev);
+ * pred[h] = sum over i ascending of q_i * C[i][h].  hot = the P experts with
+ * the largest forecast, ties to the lower index. */
+void oracle_popularity_forecast(const float* pop_prev, const int32_t* C, int E, int k_prev,
+                                int k_next, float* pred, int P, int32_t* hot) {
+    double* q = (double*)malloc(sizeof(double) * (size_t)E);
+    unsigned char* taken = (unsigned char*)calloc((size_t)E, 1);
+    if (!q || !taken) { free(q); free(taken); return; }
+    for (int i = 0; i < E; ++i) {
+        int64_t s = 0;
+        for (int h = 0; h < E; ++h) s += C[(int64_t)i * E + h];
+        q[i] = s == 0 ? 0.0
+                      : ((double)pop_prev[i] * (double)k_next) / ((double)s * (double)k_prev);
+    }
+    for (int h = 0; h < E; ++h) {
+        double a = 0.0;
+        for (int i = 0; i < E; ++i) a += q[i] * (double)C[(int64_t)i * E + h];
+        pred[h] = (float)a;
+    }
+    for (int p = 0; p < P; ++p) {
+        int best = -1;
+        for (int h = 0; h < E; ++h) {
+            if (taken[h]) continue;
+            if (best < 0 || pred[h] > pred[best]) best = h;
+        }
+        taken[best] = 1;
+        hot[p] = best;
+    }
+    free(q);
+    free(taken);
 }

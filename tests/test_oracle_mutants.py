@@ -39,6 +39,12 @@ MUTANTS = {
                           "if (best < 0 || sum[e] >= sum[best]) best = e;"),
     "bf16_double_rounding": ("double a = fabs(v);", "double a = (double)(float)fabs(v);"),
     "bf16_ties_away": ("double r = rint(ldexp(a, -q));", "double r = round(ldexp(a, -q));"),
+    "corr_transposed": ("C[(int64_t)i * E + h] += 1;", "C[(int64_t)h * E + i] += 1;"),
+    "corr_first_choice_only": ("for (int b = 0; b < k_next; ++b) {",
+                               "for (int b = 0; b < 1; ++b) {"),
+    "forecast_no_k_prev": ("((double)s * (double)k_prev)", "((double)s)"),
+    "forecast_column_sum": ("a += q[i] * (double)C[(int64_t)i * E + h];",
+                            "a += q[i] * (double)C[(int64_t)h * E + i];"),
 }
 
 

@@ -390,3 +390,71 @@ def test_ffn_hidden_activation_is_stored_at_storage_precision(dtype, eps, y_bits
         assert H.tolist() == [[1.0] * F]
         assert Yp.tolist() == [[3.0] * d]
         assert float(np.float32(3.0 + 3.0 * eps)) != 3.0
+
+
+# ------------------------------------------- cross-layer correlation forecast --
+def test_correlation_golden():
+    g = _golden("correlation_example.json")
+    C = np.zeros((g["E"], g["E"]), np.int32)
+    oracle.correlation_update(np.array(g["ids_prev"]), np.array(g["ids_next"]), C)
+    assert C.tolist() == g["C"]
+    pred, hot = oracle.popularity_forecast(np.array(g["pop_prev"]), C, g["k_prev"],
+                                           g["k_next"], 2)
+    assert pred.tolist() == g["pred"] and hot.tolist() == g["hot_P2"]
+    pred, _ = oracle.popularity_forecast(np.array(g["same_batch_pop"]), C, g["k_prev"],
+                                         g["k_next"], 0)
+    assert pred.tolist() == g["same_batch_pred"]
+
+
+def _layer_ids(rng, T, E, k):
+    return np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+
+
+@pytest.mark.parametrize("E,k_prev,k_next", [(8, 2, 2), (16, 1, 3), (5, 5, 1), (32, 4, 8)])
+def test_correlation_counts_brute_force_and_accumulate(E, k_prev, k_next):
+    rng = np.random.default_rng(E * 10 + k_prev)
+    T = 157
+    a, b = _layer_ids(rng, T, E, k_prev), _layer_ids(rng, T, E, k_next)
+    C = np.full((E, E), 3, np.int32)  # accumulates into what is there
+    oracle.correlation_update(a, b, C)
+    ref = np.full((E, E), 3, np.int64)
+    for t in range(T):
+        for i in a[t]:
+            for h in b[t]:
+                ref[i, h] += 1
+    assert np.array_equal(C, ref)
+
+
+@pytest.mark.parametrize("E,k_prev,k_next", [(8, 2, 2), (16, 1, 3), (12, 3, 1), (64, 2, 4)])
+def test_forecast_from_same_batch_reproduces_next_layer_counts(E, k_prev, k_next):
+    # With pop_prev the same batch's previous-layer counts, the forecast is
+    # exactly the next layer's counts: sum_i C[i][h] = k_prev * counts_next[h].
+    rng = np.random.default_rng(E + 7 * k_next)
+    T = 400
+    a, b = _layer_ids(rng, T, E, k_prev), _layer_ids(rng, T, E, k_next)
+    C = np.zeros((E, E), np.int32)
+    oracle.correlation_update(a, b, C)
+    counts_prev = np.bincount(a.ravel(), minlength=E).astype(np.float32)
+    counts_next = np.bincount(b.ravel(), minlength=E)
+    pred, _ = oracle.popularity_forecast(counts_prev, C, k_prev, k_next, 0)
+    np.testing.assert_allclose(pred, counts_next, rtol=2e-7)
+
+
+def test_forecast_is_linear_and_ignores_unseen_rows():
+    rng = np.random.default_rng(3)
+    E, T = 10, 200
+    a = _layer_ids(rng, T, E - 2, 2)  # experts 8 and 9 never chosen at layer j
+    b = _layer_ids(rng, T, E, 2)
+    C = np.zeros((E, E), np.int32)
+    oracle.correlation_update(a, b, C)
+    p1 = rng.uniform(0, 5, E).astype(np.float32)
+    p2 = rng.uniform(0, 5, E).astype(np.float32)
+    f1, _ = oracle.popularity_forecast(p1, C, 2, 2, 0)
+    f2, _ = oracle.popularity_forecast(p2, C, 2, 2, 0)
+    f12, _ = oracle.popularity_forecast(p1 + p2, C, 2, 2, 0)
+    np.testing.assert_allclose(f12, f1 + f2, rtol=1e-5)
+    bump = p1.copy()
+    bump[8:] += 100.0  # popularity on rows with no observed pairs adds nothing
+    fb, _ = oracle.popularity_forecast(bump, C, 2, 2, 0)
+    assert np.array_equal(fb, f1)
+    np.testing.assert_allclose(f1.sum(), p1[:8].sum(), rtol=1e-5)  # k_next / k_prev = 1
