@@ -414,6 +414,40 @@ def main():
         t = torch.tensor([e2e_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
+    # ---- next-row kernels: cross-layer correlation + popularity forecast ----
+    # Batches 0 and 1 stand for two consecutive layers of the same tokens.
+    extras = {}
+    if rank == 0:
+        ids_a = torch.empty_like(layer.ids)
+        step(0)
+        ids_a.copy_(layer.ids)
+        step(1 % nb)
+        C = torch.zeros(w.E, w.E, dtype=torch.int32, device="cuda")
+        pred = torch.empty(w.E, device="cuda")
+        hot_f = torch.empty(max(w.P, 1), dtype=torch.int32, device="cuda")
+        reps = 200
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        for _ in range(3):
+            moe.moe_correlation_update(ids_a, layer.ids, C)
+            moe.moe_popularity_forecast(layer.mean, C, w.k, w.k, pred, w.P, hot_f)
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for _ in range(reps):
+            moe.moe_correlation_update(ids_a, layer.ids, C)
+        ev[1].record(stream)
+        for _ in range(reps):
+            moe.moe_popularity_forecast(layer.mean, C, w.k, w.k, pred, w.P, hot_f)
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        corr_ms = ev[0].elapsed_time(ev[1]) / reps
+        fc_ms = ev[1].elapsed_time(ev[2]) / reps
+        corr_bytes = 2 * w.T * w.k * 4 + 2 * w.E * w.E * 4
+        extras = {
+            "correlation_update": {"ms": corr_ms, "pairs": w.T * w.k * w.k,
+                                   "gbs": corr_bytes / (corr_ms * 1e-3) / 1e9},
+            "popularity_forecast": {"ms": fc_ms, "E": w.E},
+            "note": "timed separately (200 back-to-back launches each), outside the step",
+        }
     dev_err = moe.moe_device_error()
 
     if rank == 0:
@@ -481,7 +515,7 @@ def main():
                            else "kernels issued one by one (programmatic dependent launch)",
                            "stages_and_roofline": f"{stage_steps} steps issued stage by stage, "
                                                   "events between stages"},
-                "device_error_bits": dev_err}
+                "extras": extras, "device_error_bits": dev_err}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -64,8 +64,9 @@ enum moe_dtype { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
 enum moe_device_error_bits {
     MOE_DEVERR_ROW_INDEX = 1, /* a slot_row / row_slot entry outside [0, R_max) */
     MOE_DEVERR_OFFSETS = 2,   /* offsets not non-decreasing or beyond R_max      */
-    MOE_DEVERR_TIMEOUT = 4    /* a pipeline wait inside a kernel ran past its
+    MOE_DEVERR_TIMEOUT = 4,   /* a pipeline wait inside a kernel ran past its
                                  time limit; the kernel gave up and returned     */
+    MOE_DEVERR_EXPERT_INDEX = 8 /* an expert id outside [0, E) was skipped       */
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -214,6 +215,36 @@ MOE_API int moe_popularity_update(const int32_t* counts, int E, int32_t* hist, i
  * the window on every replay.  A negative *step makes the call a no-op. */
 MOE_API int moe_popularity_update_dev(const int32_t* counts, int E, int32_t* hist, int W, int64_t* step,
                               float* mean, int P, int32_t* hot, moe_stream_t stream);
+
+/* ------------------------------------------------------------- next ----
+ * Cross-layer expert correlation.  PopFetcher, section 4.1 (Fig. 6): a
+ * token's expert choices at two consecutive MoE layers form a correlated pair.
+ * Adds, for every token t, one to C[i][h] for each i in ids_prev[t][0..k_prev)
+ * and each h in ids_next[t][0..k_next).
+ *   ids_prev [T, k_prev], ids_next [T, k_next] int32 (e.g. moe_route's ids of
+ *   layers j and j+1 for the same tokens); C [E, E] int32, accumulated into
+ *   (clear it to start a new window).  Ids outside [0, E) are skipped and
+ *   flagged (MOE_DEVERR_EXPERT_INDEX).  Deterministic (integer sums).
+ */
+MOE_API int moe_correlation_update(const int32_t* ids_prev, int k_prev, const int32_t* ids_next,
+                                   int k_next, int T, int E, int32_t* C, moe_stream_t stream);
+
+/* Correlation-based popularity forecast of the next layer.  PopFetcher,
+ * section 4.2 (Eq. 2-3, lost in extraction; read as below):
+ *   P(h|i)  = C[i][h] / n_i,  n_i = (sum_h C[i][h]) / k_next
+ *   pred[h] = sum_i pop_prev[i] * P(h|i) / k_prev
+ * evaluated in IEEE double as q_i = (pop_prev[i] * k_next) / (S_i * k_prev)
+ * (S_i = sum_h C[i][h]; q_i = 0 when S_i = 0), pred[h] = sum_i q_i * C[i][h]
+ * with i ascending, each operation rounded separately, rounded once to fp32.
+ * hot [P]: the P largest forecasts, equal values to the lower index.
+ *   pop_prev [E] fp32 (e.g. moe_popularity_update's window mean of layer j);
+ *   C [E, E] from moe_correlation_update; pred [E] fp32; 0 <= P <= E.
+ * With pop_prev = layer j's counts and C from the same batch, pred equals
+ * layer j+1's counts.
+ */
+MOE_API int moe_popularity_forecast(const float* pop_prev, const int32_t* C, int E, int k_prev,
+                                    int k_next, float* pred, int P, int32_t* hot,
+                                    moe_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -25,6 +25,7 @@ MOE_DTYPE_BF16 = 1
 MOE_DEVERR_ROW_INDEX = 1
 MOE_DEVERR_OFFSETS = 2
 MOE_DEVERR_TIMEOUT = 4
+MOE_DEVERR_EXPERT_INDEX = 8
 
 _p, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
 _SIGS = {
@@ -40,6 +41,8 @@ _SIGS = {
     "moe_popularity_update": ([_p, _i, _p, _i, _i64, _p, _i, _p, _p], _i),
     "moe_popularity_update_dev": ([_p, _i, _p, _i, _p, _p, _i, _p, _p], _i),
     "moe_route_noalloc": ([_p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i),
+    "moe_correlation_update": ([_p, _i, _p, _i, _i, _i, _p, _p], _i),
+    "moe_popularity_forecast": ([_p, _p, _i, _i, _i, _p, _i, _p, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -144,6 +147,19 @@ def moe_route_noalloc(logits, bias, k, capacity, ids, w, counts, kept, offsets, 
     _check("moe_route_noalloc", lib.moe_route_noalloc(
         _ptr(logits), _ptr(bias), T, E, k, int(capacity), _ptr(ids), _ptr(w), _ptr(counts),
         _ptr(kept), _ptr(offsets), _ptr(slot_row), _ptr(row_slot), _ptr(n_dropped),
+        _stream(stream)))
+
+
+def moe_correlation_update(ids_prev, ids_next, C, stream=None):
+    T, k_prev = ids_prev.shape
+    _check("moe_correlation_update", lib.moe_correlation_update(
+        _ptr(ids_prev), k_prev, _ptr(ids_next), ids_next.shape[1], T, C.shape[0], _ptr(C),
+        _stream(stream)))
+
+
+def moe_popularity_forecast(pop_prev, C, k_prev, k_next, pred, P, hot, stream=None):
+    _check("moe_popularity_forecast", lib.moe_popularity_forecast(
+        _ptr(pop_prev), _ptr(C), C.shape[0], k_prev, k_next, _ptr(pred), P, _ptr(hot),
         _stream(stream)))
 
 

@@ -55,7 +55,8 @@ def test_route_workspace_size(lib):
     lib.moe_route_workspace_size.restype = ctypes.c_size_t
     f = lib.moe_route_workspace_size
     assert f(0, 8, 2) >= 256
-    assert f(4096, 16, 2) >= 2 * 32 * 16 * 4
+    assert f(4096, 16, 2) >= 2 * 16 * 16 * 4  # two int32 [chunk][expert] tables
+    assert f(8192, 16, 2) > f(4096, 16, 2) and f(4096, 64, 2) > f(4096, 16, 2)
     assert f(-1, 8, 2) == 0
 
 
