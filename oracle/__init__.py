@@ -74,6 +74,8 @@ def _load():
         lib.oracle_correlation_update.restype = None
         lib.oracle_popularity_forecast.argtypes = [p, p, i32, i32, i32, p, i32, p]
         lib.oracle_popularity_forecast.restype = None
+        lib.oracle_aux_loss.argtypes = [p, p, i32, i32, i32, p, p]
+        lib.oracle_aux_loss.restype = ctypes.c_float
         lib.oracle_round_bf16.argtypes = [ctypes.c_double]
         lib.oracle_round_bf16.restype = ctypes.c_uint16
         _lib = lib
@@ -232,6 +234,17 @@ def popularity_forecast(pop_prev: np.ndarray, C: np.ndarray, k_prev: int, k_next
     _load().oracle_popularity_forecast(_ptr(pop), _ptr(Cc), E, k_prev, k_next, _ptr(pred), P,
                                        _ptr(hot))
     return pred, hot[:P].copy()
+
+
+def aux_loss(logits: np.ndarray, bias, k: int, counts: np.ndarray):
+    """GShard balancing loss E * sum_e f_e P_e; returns (loss fp32, P_e [E] fp32)."""
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    b = None if bias is None else _c(bias, np.float32)
+    cnt = _c(counts, np.int32)
+    P = np.empty(E, np.float32)
+    loss = _load().oracle_aux_loss(_ptr(lg), _ptr(b), T, E, k, _ptr(cnt), _ptr(P))
+    return np.float32(loss), P
 
 
 def layer(x, Wg, W1, W2, bias, k, capacity=0, logits=None):

@@ -33,6 +33,8 @@
  *   [Pop-4.2b]  PopFetcher, section 4.2, Eq. 2-3 (lost): the conditional
  *               probability of the next-layer expert given the previous-layer
  *               one, and the correlation-based popularity forecast.
+ *   [Pop-2.3.1] PopFetcher, section 2.3.1: GShard adds a load-balancing loss to
+ *               spread the workload evenly (formula not on the pages).
  *   [MPMC]      MoE-MPMC summary, problem statement item 3: routing is softmax
  *               based.
  *
@@ -390,4 +392,46 @@ void oracle_popularity_forecast(const float* pop_prev, const int32_t* C, int E, 
     }
     free(q);
     free(taken);
+}
+
+/* ----------------------------------------------- load-balancing loss (f4) -- */
+
+/* GShard's auxiliary load-balancing loss.  PopFetcher, section 2.3.1, names it
+ * (GShard spreads the workload evenly across workers with a balancing loss)
+ * without the formula; reading taken (GShard / Switch form):
+ *   f_e  = counts[e] / (T * k)          fraction of routed slots on expert e
+ *   P_e  = (1/T) sum_t softmax(z_t)_e   mean router probability of expert e,
+ *          z = logits + bias (one fp32 add, the routing keys)
+ *   loss = E * sum_e f_e * P_e          (= 1 when routing and probabilities
+ *                                         are both uniform)
+ * In double, e ascending; loss and the P_e rounded once to fp32. */
+float oracle_aux_loss(const float* logits, const float* bias, int T, int E, int k,
+                      const int32_t* counts, float* prob_mean) {
+    double* P = (double*)calloc((size_t)E, sizeof(double));
+    double* ex = (double*)malloc(sizeof(double) * (size_t)E);
+    if (!P || !ex) { free(P); free(ex); return NAN; }
+    for (int t = 0; t < T; ++t) {
+        double zmax = -INFINITY;
+        for (int e = 0; e < E; ++e) {
+            float z = logits[(int64_t)t * E + e] + (bias ? bias[e] : 0.0f);
+            ex[e] = (double)z;
+            if (ex[e] > zmax) zmax = ex[e];
+        }
+        double D = 0.0;
+        for (int e = 0; e < E; ++e) {
+            ex[e] = exp(ex[e] - zmax);
+            D += ex[e];
+        }
+        for (int e = 0; e < E; ++e) P[e] += ex[e] / D;
+    }
+    double loss = 0.0;
+    for (int e = 0; e < E; ++e) {
+        double Pe = T > 0 ? P[e] / (double)T : 0.0;
+        double fe = T > 0 ? (double)counts[e] / ((double)T * (double)k) : 0.0;
+        loss += fe * Pe;
+        if (prob_mean) prob_mean[e] = (float)Pe;
+    }
+    free(P);
+    free(ex);
+    return (float)((double)E * loss);
 }

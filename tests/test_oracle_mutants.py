@@ -43,6 +43,12 @@ MUTANTS = {
     "corr_first_choice_only": ("for (int b = 0; b < k_next; ++b) {",
                                "for (int b = 0; b < 1; ++b) {"),
     "forecast_no_k_prev": ("((double)s * (double)k_prev)", "((double)s)"),
+    "aux_bias_ignored": ("float z = logits[(int64_t)t * E + e] + (bias ? bias[e] : 0.0f);",
+                         "float z = logits[(int64_t)t * E + e];"),
+    "aux_f_not_over_k": ("(double)counts[e] / ((double)T * (double)k)",
+                         "(double)counts[e] / (double)T"),
+    "aux_unnormalised_softmax": ("for (int e = 0; e < E; ++e) P[e] += ex[e] / D;",
+                                 "for (int e = 0; e < E; ++e) P[e] += ex[e];"),
     "forecast_column_sum": ("a += q[i] * (double)C[(int64_t)i * E + h];",
                             "a += q[i] * (double)C[(int64_t)h * E + i];"),
 }

@@ -458,3 +458,59 @@ def test_forecast_is_linear_and_ignores_unseen_rows():
     fb, _ = oracle.popularity_forecast(bump, C, 2, 2, 0)
     assert np.array_equal(fb, f1)
     np.testing.assert_allclose(f1.sum(), p1[:8].sum(), rtol=1e-5)  # k_next / k_prev = 1
+
+
+# ------------------------------------------------------ load-balancing loss --
+def test_aux_loss_golden():
+    g = _golden("aux_loss_example.json")
+    lg = np.array(g["logits"], np.float32)
+    r = oracle.route(lg, None, g["k"])
+    assert r["counts"].tolist() == g["counts"]
+    loss, P = oracle.aux_loss(lg, None, g["k"], r["counts"])
+    np.testing.assert_allclose(P, g["prob_mean"], rtol=1e-7)
+    np.testing.assert_allclose(loss, g["loss"], rtol=1e-7)
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (16, 1), (5, 5)])
+def test_aux_loss_uniform_router_is_one(E, k):
+    T = 96
+    lg = np.full((T, E), 0.37, np.float32)  # every probability 1/E, any routing
+    r = oracle.route(lg, None, k)
+    loss, P = oracle.aux_loss(lg, None, k, r["counts"])
+    np.testing.assert_allclose(P, 1.0 / E, rtol=1e-7)
+    np.testing.assert_allclose(loss, 1.0, rtol=1e-6)
+
+
+def test_aux_loss_is_invariant_to_relabelling_experts():
+    rng = np.random.default_rng(4)
+    T, E, k = 300, 12, 3
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    b = rng.standard_normal(E).astype(np.float32)
+    perm = rng.permutation(E)
+    r = oracle.route(lg, b, k)
+    r2 = oracle.route(lg[:, perm], b[perm], k)
+    l1, P1 = oracle.aux_loss(lg, b, k, r["counts"])
+    l2, P2 = oracle.aux_loss(lg[:, perm], b[perm], k, r2["counts"])
+    np.testing.assert_allclose(l1, l2, rtol=1e-6)
+    np.testing.assert_allclose(P1[perm], P2, rtol=1e-6)
+
+
+def test_aux_loss_collapsed_router_approaches_e():
+    T, E = 64, 8
+    lg = np.zeros((T, E), np.float32)
+    lg[:, 3] = 40.0  # softmax ~ one-hot on expert 3, every token routed there
+    r = oracle.route(lg, None, 1)
+    loss, P = oracle.aux_loss(lg, None, 1, r["counts"])
+    np.testing.assert_allclose(loss, E, rtol=1e-6)
+    np.testing.assert_allclose(P.sum(), 1.0, rtol=1e-6)
+
+
+def test_aux_loss_probabilities_include_the_routing_bias():
+    # zero logits, bias (ln 3, 0): every token has p = (3/4, 1/4) and is routed
+    # to expert 0, so loss = 2 * (1 * 3/4 + 0 * 1/4) = 1.5
+    lg = np.zeros((10, 2), np.float32)
+    b = np.array([np.log(3.0), 0.0], np.float32)
+    r = oracle.route(lg, b, 1)
+    loss, P = oracle.aux_loss(lg, b, 1, r["counts"])
+    np.testing.assert_allclose(P, [0.75, 0.25], rtol=1e-7)
+    np.testing.assert_allclose(loss, 1.5, rtol=1e-7)
