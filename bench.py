@@ -441,11 +441,30 @@ def main():
         torch.cuda.synchronize()
         corr_ms = ev[0].elapsed_time(ev[1]) / reps
         fc_ms = ev[1].elapsed_time(ev[2]) / reps
+        # GShard balancing loss of the last routing call (re-reads the logits)
+        logits_last = batches[1 % nb].get("logits")
+        if logits_last is None:
+            logits_last = layer.logits
+        aux_loss = torch.empty(1, device="cuda")
+        aux_P = torch.empty(w.E, device="cuda")
+        bias_last = batches[1 % nb]["bias"]
+        for _ in range(3):
+            moe.moe_aux_loss(logits_last, bias_last, w.k, layer.counts, aux_loss, aux_P,
+                             layer.workspace)
+        ev[0].record(stream)
+        for _ in range(reps):
+            moe.moe_aux_loss(logits_last, bias_last, w.k, layer.counts, aux_loss, aux_P,
+                             layer.workspace)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        aux_ms = ev[0].elapsed_time(ev[1]) / reps
         corr_bytes = 2 * w.T * w.k * 4 + 2 * w.E * w.E * 4
         extras = {
             "correlation_update": {"ms": corr_ms, "pairs": w.T * w.k * w.k,
                                    "gbs": corr_bytes / (corr_ms * 1e-3) / 1e9},
             "popularity_forecast": {"ms": fc_ms, "E": w.E},
+            "aux_loss": {"ms": aux_ms, "value": float(aux_loss.item()),
+                         "gbs": w.T * w.E * 4 / (aux_ms * 1e-3) / 1e9},
             "note": "timed separately (200 back-to-back launches each), outside the step",
         }
     dev_err = moe.moe_device_error()

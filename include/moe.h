@@ -246,6 +246,21 @@ MOE_API int moe_popularity_forecast(const float* pop_prev, const int32_t* C, int
                                     int k_next, float* pred, int P, int32_t* hot,
                                     moe_stream_t stream);
 
+/* GShard load-balancing loss of one routing call.  PopFetcher, section 2.3.1
+ * names it (it evens out the workload across workers); the formula is not on
+ * the pages and is read as the GShard / Switch form:
+ *   f_e = counts[e] / (T k),  P_e = mean_t softmax(logits[t] + bias)_e,
+ *   loss = E * sum_e f_e P_e   (1 for a uniform router, E for a collapsed one)
+ *   logits [T,E] fp32, bias [E] or NULL (the same keys moe_route ranked);
+ *   counts [E] from moe_route; loss [1] fp32; prob_mean [E] fp32 or NULL.
+ *   workspace: at least moe_route_workspace_size(T, E, k) bytes (the router's
+ *   workspace can be reused once moe_route's kernels are done).
+ * fp32 softmax per token, sums in a fixed order (deterministic).
+ */
+MOE_API int moe_aux_loss(const float* logits, const float* bias, int T, int E, int k,
+                         const int32_t* counts, float* loss, float* prob_mean, void* workspace,
+                         size_t workspace_bytes, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

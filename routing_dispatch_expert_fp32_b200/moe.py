@@ -43,6 +43,7 @@ _SIGS = {
     "moe_route_noalloc": ([_p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i),
     "moe_correlation_update": ([_p, _i, _p, _i, _i, _i, _p, _p], _i),
     "moe_popularity_forecast": ([_p, _p, _i, _i, _i, _p, _i, _p, _p], _i),
+    "moe_aux_loss": ([_p, _p, _i, _i, _i, _p, _p, _p, _p, _sz, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -161,6 +162,13 @@ def moe_popularity_forecast(pop_prev, C, k_prev, k_next, pred, P, hot, stream=No
     _check("moe_popularity_forecast", lib.moe_popularity_forecast(
         _ptr(pop_prev), _ptr(C), C.shape[0], k_prev, k_next, _ptr(pred), P, _ptr(hot),
         _stream(stream)))
+
+
+def moe_aux_loss(logits, bias, k, counts, loss, prob_mean, workspace, stream=None):
+    T, E = logits.shape
+    _check("moe_aux_loss", lib.moe_aux_loss(
+        _ptr(logits), _ptr(bias), T, E, k, _ptr(counts), _ptr(loss), _ptr(prob_mean),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 class MoELayer:
