@@ -85,7 +85,7 @@ def load_peaks():
 GEMM_SOURCES = ["gemm_tc.cu", "grouped.cuh", "common.cuh"]
 
 
-def gemm_traffic(workload: str):
+def gemm_traffic(workload: str, kernel: str):
     """Measured DRAM bytes per launch of the grouped GEMM from profiles/traffic.md,
     or None when missing or taken on different kernel sources."""
     import hashlib
@@ -99,7 +99,7 @@ def gemm_traffic(workload: str):
         return None
     for line in open(path):
         cells = [c.strip() for c in line.strip().strip("|").split("|")]
-        if len(cells) == 4 and cells[0] == workload and cells[3] == sha:
+        if len(cells) == 4 and cells[0] == workload and cells[1] == kernel and cells[3] == sha:
             try:
                 return int(cells[2])
             except ValueError:
@@ -503,16 +503,22 @@ def main():
         else:
             # the grouped GEMM: two launches per step, 2*R*d*F flops each
             launch_ms = per["expert_ffn"]["ms"] / 2
-            roof = {"bound": "tensor", "kernel": "gemm_tc_kernel",
+            # the library takes 2-CTA pair tiles when R_max / E >= 1024
+            pair = w.dtype == "bf16" and w.T * w.k >= 1024 * w.E
+            roof = {"bound": "tensor", "kernel": "gemm_tc2_kernel" if pair else "gemm_tc_kernel",
                     "achieved": 2.0 * R_mean * w.d * w.F / (launch_ms * 1e-3) / 1e12,
                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
             if w.dtype == "f32":
+                # fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x the max SM clock
                 roof["bound"] = "alu"
                 roof["kernel"] = "gemm_simt_f32_kernel"
+                roof["peak"] = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
         roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["peak_source"] = f"{peak_src} ({'bf16_tflops_sustained' if roof['unit'] == 'TFLOP/s' else 'hbm_gbs'})"
-        roof["traffic"] = (gemm_traffic(w.name)
-                           if roof["kernel"] == "gemm_tc_kernel" and args.tokens == 0
+        roof["peak_source"] = (
+            "derived fp32 FMA peak: 148 x 128 x 2 x sm_max_mhz" if roof["bound"] == "alu" else
+            f"{peak_src} ({'bf16_tflops_sustained' if roof['unit'] == 'TFLOP/s' else 'hbm_gbs'})")
+        roof["traffic"] = (gemm_traffic(w.name, roof["kernel"])
+                           if roof["kernel"].startswith("gemm_tc") and args.tokens == 0
                            and args.experts == 0 else None)
         value = w.T * steps * world / (elapsed_ms * 1e-3)
         cpu = None

@@ -6,7 +6,7 @@
 // encode.  bf16 layers run on the tcgen05 tensor cores; fp32 layers on the
 // CUDA cores (fp32 products, no TF32).  The gate projection (PopFetcher,
 // section 2.1.2) is the same GEMM with one group and fp32 output, or, for
-// E <= 32, the skinny CUDA-core kernel of gate.cu.
+// fp32 layers with E <= 32, the skinny CUDA-core kernel of gate.cu.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -47,7 +47,11 @@ extern "C" MOE_API int moe_gate(const void* x, const void* Wg, int dtype, int T,
     if ((d * dtype_bytes(dtype)) % 16 != 0) return MOE_ERR_UNSUPPORTED;
     if (!aligned16(x) || !aligned16(Wg) || !aligned16(logits)) return MOE_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (gate_small_fits(E, d, dtype)) return launch_gate_small(x, Wg, dtype, T, d, E, logits, st);
+    // fp32 layers with few experts: the CUDA-core kernel (measured faster than
+    // the tiled SIMT GEMM there); bf16 stays on the tensor cores, which were
+    // measured faster than that kernel.
+    if (dtype == MOE_DTYPE_F32 && gate_small_fits(E, d, dtype))
+        return launch_gate_small(x, Wg, dtype, T, d, E, logits, st);
     if (dtype == MOE_DTYPE_BF16)
         return launch_gemm_tc_bf16(x, Wg, logits, true, E, d, 1, nullptr, T, T, false, st);
     return launch_gemm_simt_f32(static_cast<const float*>(x), static_cast<const float*>(Wg), logits,

@@ -13,8 +13,9 @@
 // for E <= 128 into a per-CTA shared-memory histogram flushed with one global
 // atomicAdd per non-zero bin, else straight into global memory.  Integer sums
 // commute, so the result does not depend on the order.
-// moe_popularity_forecast: one CTA.  Row sums S_i (a warp per row), then
-// q_i = (pop_i * k_next) / (S_i * k_prev) and pred[h] = sum_i q_i * C[i][h] in
+// moe_popularity_forecast: one CTA of 1024 threads.  Row sums S_i (a warp per
+// row), then q_i = (pop_i * k_next) / (S_i * k_prev) and, with C streamed
+// through shared memory in row chunks, pred[h] = sum_i q_i * C[i][h] in
 // IEEE double with every operation rounded separately (no fused multiply-add),
 // i ascending, rounded once to fp32: bit-identical to the same sequence of
 // operations done anywhere else.  Hot experts: rank by (pred desc, index asc).
@@ -64,15 +65,20 @@ correlation_kernel(const int32_t* __restrict__ ids_prev, int k_prev,
     }
 }
 
-__global__ void __launch_bounds__(1024)
+constexpr int kForecastThreads = 1024;
+constexpr int kForecastStage = 8192;  // int32 counters staged per pass (32 KB)
+
+__global__ void __launch_bounds__(kForecastThreads)
 forecast_kernel(const float* __restrict__ pop_prev, const int32_t* __restrict__ C, int E,
                 int k_prev, int k_next, float* __restrict__ pred, int P, int32_t* __restrict__ hot) {
     __shared__ double s_q[kMaxExperts];
     __shared__ float s_pred[kMaxExperts];
+    __shared__ int32_t s_c[kForecastStage];
     pdl_wait();
     pdl_trigger();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    for (int i = warp; i < E; i += nwarps) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kWarps = kForecastThreads / 32;
+    for (int i = warp; i < E; i += kWarps) {
         long long s = 0;
         for (int h = lane; h < E; h += 32) s += C[(size_t)i * E + h];
 #pragma unroll
@@ -83,16 +89,27 @@ forecast_kernel(const float* __restrict__ pop_prev, const int32_t* __restrict__ 
             s_q[i] = s == 0 ? 0.0 : __ddiv_rn(num, den);
         }
     }
-    __syncthreads();
-    for (int h = threadIdx.x; h < E; h += blockDim.x) {
-        double a = 0.0;
-        for (int i = 0; i < E; ++i) a = __dadd_rn(a, __dmul_rn(s_q[i], (double)C[(size_t)i * E + h]));
-        const float f = __double2float_rn(a);
-        pred[h] = f;
-        s_pred[h] = f;
+    // pred[h] = sum over i ascending of q_i * C[i][h]; rows of C pass through
+    // shared memory in chunks, each thread owning columns h = tid, tid + 1024
+    const int rows_per_pass = kForecastStage / E;
+    double acc = 0.0;  // thread's column h = tid (E <= 1024)
+    for (int i0 = 0; i0 < E; i0 += rows_per_pass) {
+        const int i1 = min(E, i0 + rows_per_pass);
+        __syncthreads();  // s_q ready (first pass) / previous chunk consumed
+        for (int idx = tid; idx < (i1 - i0) * E; idx += kForecastThreads)
+            s_c[idx] = C[(size_t)i0 * E + idx];
+        __syncthreads();
+        if (tid < E)
+            for (int i = i0; i < i1; ++i)
+                acc = __dadd_rn(acc, __dmul_rn(s_q[i], (double)s_c[(i - i0) * E + tid]));
+    }
+    if (tid < E) {
+        const float f = __double2float_rn(acc);
+        pred[tid] = f;
+        s_pred[tid] = f;
     }
     __syncthreads();
-    for (int h = threadIdx.x; h < E; h += blockDim.x) {
+    for (int h = tid; h < E; h += kForecastThreads) {
         const float mine = s_pred[h];
         int rank = 0;
         for (int o = 0; o < E; ++o) {
@@ -138,7 +155,7 @@ extern "C" MOE_API int moe_popularity_forecast(const float* pop_prev, const int3
     if (E < 1 || E > kMaxExperts || k_prev < 1 || k_next < 1 || P < 0 || P > E)
         return MOE_ERR_INVALID_ARG;
     if (!pop_prev || !C || !pred || (P > 0 && !hot)) return MOE_ERR_INVALID_ARG;
-    const int threads = E < 32 ? 32 : (E > 1024 ? 1024 : ((E + 31) / 32) * 32);
-    return launch_pdl(forecast_kernel, 1, threads, 0, reinterpret_cast<cudaStream_t>(stream),
-                      pop_prev, C, E, k_prev, k_next, pred, P, hot);
+    return launch_pdl(forecast_kernel, 1, kForecastThreads, 0,
+                      reinterpret_cast<cudaStream_t>(stream), pop_prev, C, E, k_prev, k_next, pred,
+                      P, hot);
 }
