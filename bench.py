@@ -276,11 +276,12 @@ def main():
     if world > 1:
         hook = lambda c: dist.all_reduce(c)  # noqa: E731  global popularity (sum over ranks)
 
-    def step(i, ev=None):
+    def step(i, ev=None, collective=True):
         b = batches[i % nb]
         if ev is None:
             layer.forward(b["x"], weights.get("Wg"), weights.get("W1"), weights.get("W2"),
-                          b["bias"], logits=b.get("logits"), counts_hook=hook)
+                          b["bias"], logits=b.get("logits"),
+                          counts_hook=hook if collective else None)
             return
         # same calls as MoELayer.forward, with an event after each stage
         ev[0].record(stream)
@@ -419,9 +420,9 @@ def main():
     extras = {}
     if rank == 0:
         ids_a = torch.empty_like(layer.ids)
-        step(0)
+        step(0, collective=False)  # rank 0 only: no collective here
         ids_a.copy_(layer.ids)
-        step(1 % nb)
+        step(1 % nb, collective=False)
         C = torch.zeros(w.E, w.E, dtype=torch.int32, device="cuda")
         pred = torch.empty(w.E, device="cuda")
         hot_f = torch.empty(max(w.P, 1), dtype=torch.int32, device="cuda")

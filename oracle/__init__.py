@@ -76,6 +76,17 @@ def _load():
         lib.oracle_popularity_forecast.restype = None
         lib.oracle_aux_loss.argtypes = [p, p, i32, i32, i32, p, p]
         lib.oracle_aux_loss.restype = ctypes.c_float
+        lib.oracle_combine_backward.argtypes = [p, p, i32, i32, i32, i32, p, p, p, p]
+        lib.oracle_combine_backward.restype = None
+        lib.oracle_expert_ffn_backward.argtypes = [p, p, p, p, p, i32, i32, i32, i32, p, p, p, p,
+                                                   p]
+        lib.oracle_expert_ffn_backward.restype = None
+        lib.oracle_dispatch_backward.argtypes = [p, i32, i32, i32, i32, p, p]
+        lib.oracle_dispatch_backward.restype = None
+        lib.oracle_route_backward.argtypes = [p, p, p, i32, i32, i32, p, p]
+        lib.oracle_route_backward.restype = None
+        lib.oracle_gate_backward.argtypes = [p, p, i32, i32, i32, i32, p, p, p]
+        lib.oracle_gate_backward.restype = None
         lib.oracle_round_bf16.argtypes = [ctypes.c_double]
         lib.oracle_round_bf16.restype = ctypes.c_uint16
         _lib = lib
@@ -247,12 +258,84 @@ def aux_loss(logits: np.ndarray, bias, k: int, counts: np.ndarray):
     return np.float32(loss), P
 
 
+def combine_backward(dy, Yp, k, slot_row, w):
+    """(dw [T,k] fp32, dYp [rows(Yp), d] dtype; rows no slot names stay zero)."""
+    dy, Yp = _c(dy), _c(Yp)
+    dt = _dtype_code(dy)
+    T, d = dy.shape
+    sr, ww = _c(slot_row, np.int32), _c(w, np.float32)
+    dw = np.empty((T, k), np.float32)
+    dYp = np.zeros_like(Yp)
+    _load().oracle_combine_backward(_ptr(dy), _ptr(Yp), dt, T, d, k, _ptr(sr), _ptr(ww), _ptr(dw),
+                                    _ptr(dYp))
+    return dw, dYp
+
+
+def expert_ffn_backward(Xp, H, dYp, W1, W2, offsets):
+    """(dH, dXp, dW1 fp32 [E,F,d], dW2 fp32 [E,d,F]) over the grouped rows."""
+    Xp, H, dYp, W1, W2 = _c(Xp), _c(H), _c(dYp), _c(W1), _c(W2)
+    dt = _dtype_code(Xp)
+    E, F, d = W1.shape
+    off = _c(offsets, np.int32)
+    dH = np.zeros_like(H)
+    dXp = np.zeros_like(Xp)
+    dW1 = np.zeros((E, F, d), np.float32)
+    dW2 = np.zeros((E, d, F), np.float32)
+    _load().oracle_expert_ffn_backward(_ptr(Xp), _ptr(H), _ptr(dYp), _ptr(W1), _ptr(W2), dt, E, d,
+                                       F, _ptr(off), _ptr(dH), _ptr(dXp), _ptr(dW1), _ptr(dW2))
+    return dH, dXp, dW1, dW2
+
+
+def dispatch_backward(dXp, T, k, slot_row):
+    dXp = _c(dXp)
+    dt = _dtype_code(dXp)
+    d = dXp.shape[1]
+    dx = np.empty((T, d), dXp.dtype)
+    _load().oracle_dispatch_backward(_ptr(dXp), dt, T, d, k, _ptr(_c(slot_row, np.int32)),
+                                     _ptr(dx))
+    return dx
+
+
+def route_backward(ids, w, dw, E):
+    """(dlogits [T,E] fp32, dbias [E] fp32)."""
+    ids, w, dw = _c(ids, np.int32), _c(w, np.float32), _c(dw, np.float32)
+    T, k = ids.shape
+    dl = np.empty((T, E), np.float32)
+    db = np.empty(E, np.float32)
+    _load().oracle_route_backward(_ptr(ids), _ptr(w), _ptr(dw), T, E, k, _ptr(dl), _ptr(db))
+    return dl, db
+
+
+def gate_backward(x, Wg, dlogits, dx):
+    """Adds the gate's input gradient into a copy of dx; returns (dx, dWg fp32)."""
+    x, Wg = _c(x), _c(Wg)
+    dt = _dtype_code(x)
+    T, d = x.shape
+    E = Wg.shape[0]
+    dx = np.array(dx, copy=True)
+    dWg = np.empty((E, d), np.float32)
+    _load().oracle_gate_backward(_ptr(x), _ptr(Wg), dt, T, d, E, _ptr(_c(dlogits, np.float32)),
+                                 _ptr(dx), _ptr(dWg))
+    return dx, dWg
+
+
+def layer_backward(x, Wg, W1, W2, bias, k, fwd, dy):
+    """Whole-layer backward from the forward record `fwd` (layer(..., want_h) output)."""
+    dw, dYp = combine_backward(dy, fwd["Yp"], k, fwd["slot_row"], fwd["w"])
+    dH, dXp, dW1, dW2 = expert_ffn_backward(fwd["Xp"], fwd["H"], dYp, W1, W2, fwd["offsets"])
+    dx = dispatch_backward(dXp, x.shape[0], k, fwd["slot_row"])
+    dlogits, dbias = route_backward(fwd["ids"], fwd["w"], dw, Wg.shape[0])
+    dx, dWg = gate_backward(x, Wg, dlogits, dx)
+    return dict(dw=dw, dYp=dYp, dH=dH, dXp=dXp, dW1=dW1, dW2=dW2, dlogits=dlogits,
+                dbias=dbias, dx=dx, dWg=dWg)
+
+
 def layer(x, Wg, W1, W2, bias, k, capacity=0, logits=None):
     """Whole layer: gate (unless logits are given), route, dispatch, FFN, combine."""
     if logits is None:
         logits = gate(x, Wg)
     r = route(logits, bias, k, capacity)
     Xp = dispatch(x, k, r["row_slot"])
-    Yp = expert_ffn(Xp, W1, W2, r["offsets"])
+    Yp, H = expert_ffn(Xp, W1, W2, r["offsets"], want_h=True)
     y = combine(Yp, x.shape[0], k, r["slot_row"], r["w"])
-    return dict(logits=logits, Xp=Xp, Yp=Yp, y=y, **r)
+    return dict(logits=logits, Xp=Xp, H=H, Yp=Yp, y=y, **r)

@@ -435,3 +435,147 @@ float oracle_aux_loss(const float* logits, const float* bias, int T, int E, int 
     free(ex);
     return (float)((double)E * loss);
 }
+
+/* ------------------------------------------------------------ backward (f1) -- */
+
+/* Backward of the MoE layer (PopFetcher, section 5.2.1: every expert GEMM of
+ * the forward pass has two in the backward pass, for the input and for the
+ * weights).  Gradients of the layer as written above, taken in exact
+ * arithmetic at the stored forward values (the bf16 storage roundings of H and
+ * Yp pass the gradient through unchanged), accumulated in double and rounded
+ * once to the storage type of the tensor written.
+ *
+ * Output decode / combine:   dw[t][j]  = <dy[t], Yp[row]>            (fp32)
+ *                            dYp[row]  = w[t][j] * dy[t]             (dtype)
+ * for kept slots (row = slot_row[t][j] >= 0); dropped slots: dw = 0. */
+void oracle_combine_backward(const void* dy, const void* Yp, int dtype, int T, int d, int k,
+                             const int32_t* slot_row, const float* w, float* dw, void* dYp) {
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int64_t s = (int64_t)t * k + j;
+            int32_t row = slot_row[s];
+            if (row < 0) { dw[s] = 0.0f; continue; }
+            double dot = 0.0;
+            for (int o = 0; o < d; ++o) {
+                double g = load_elem(dy, dtype, (int64_t)t * d + o);
+                dot += g * load_elem(Yp, dtype, (int64_t)row * d + o);
+                store_elem(dYp, dtype, (int64_t)row * d + o, (double)w[s] * g);
+            }
+            dw[s] = (float)dot;
+        }
+}
+
+/* Expert computation, backward, for the rows of each group e:
+ *   dH[r][f]   = (H[r][f] > 0) ? sum_o dYp[r][o] W2[e][o][f] : 0      (ReLU)
+ *   dXp[r][c]  = sum_f dH[r][f] W1[e][f][c]
+ *   dW2[e][o][f] = sum_r dYp[r][o] H[r][f]      dW1[e][f][c] = sum_r dH[r][f] Xp[r][c]
+ * dH is stored in dtype and that stored value feeds dXp and dW1 (as on the
+ * GPU, where it is a tensor between two GEMMs).  dW1, dW2 are fp32; dH, dXp
+ * dtype.  Any of dW1 / dW2 may be NULL. */
+void oracle_expert_ffn_backward(const void* Xp, const void* H, const void* dYp, const void* W1,
+                                const void* W2, int dtype, int E, int d, int F,
+                                const int32_t* offsets, void* dH, void* dXp, float* dW1,
+                                float* dW2) {
+    double* g = (double*)malloc(sizeof(double) * (size_t)F);
+    if (!g) return;
+    for (int e = 0; e < E; ++e) {
+        const int64_t w1b = (int64_t)e * F * d, w2b = (int64_t)e * d * F;
+        for (int r = offsets[e]; r < offsets[e + 1]; ++r) {
+            for (int f = 0; f < F; ++f) {
+                double acc = 0.0;
+                if (load_elem(H, dtype, (int64_t)r * F + f) > 0.0)
+                    for (int o = 0; o < d; ++o)
+                        acc += load_elem(dYp, dtype, (int64_t)r * d + o) *
+                               load_elem(W2, dtype, w2b + (int64_t)o * F + f);
+                store_elem(dH, dtype, (int64_t)r * F + f, acc);
+                g[f] = load_elem(dH, dtype, (int64_t)r * F + f);
+            }
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int f = 0; f < F; ++f)
+                    acc += g[f] * load_elem(W1, dtype, w1b + (int64_t)f * d + c);
+                store_elem(dXp, dtype, (int64_t)r * d + c, acc);
+            }
+        }
+        if (dW2)
+            for (int o = 0; o < d; ++o)
+                for (int f = 0; f < F; ++f) {
+                    double acc = 0.0;
+                    for (int r = offsets[e]; r < offsets[e + 1]; ++r)
+                        acc += load_elem(dYp, dtype, (int64_t)r * d + o) *
+                               load_elem(H, dtype, (int64_t)r * F + f);
+                    dW2[w2b + (int64_t)o * F + f] = (float)acc;
+                }
+        if (dW1)
+            for (int f = 0; f < F; ++f)
+                for (int c = 0; c < d; ++c) {
+                    double acc = 0.0;
+                    for (int r = offsets[e]; r < offsets[e + 1]; ++r)
+                        acc += load_elem(dH, dtype, (int64_t)r * F + f) *
+                               load_elem(Xp, dtype, (int64_t)r * d + c);
+                    dW1[w1b + (int64_t)f * d + c] = (float)acc;
+                }
+    }
+    free(g);
+}
+
+/* Input encode, backward: each token's rows return to it,
+ * dx[t] = sum over kept slots of dXp[slot_row[t][j]], j ascending (dtype). */
+void oracle_dispatch_backward(const void* dXp, int dtype, int T, int d, int k,
+                              const int32_t* slot_row, void* dx) {
+    for (int t = 0; t < T; ++t)
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int32_t row = slot_row[(int64_t)t * k + j];
+                if (row >= 0) acc += load_elem(dXp, dtype, (int64_t)row * d + c);
+            }
+            store_elem(dx, dtype, (int64_t)t * d + c, acc);
+        }
+}
+
+/* Gate routing, backward.  w_j = exp(z_j) / sum_{i in S_t} exp(z_i) over the
+ * token's selected experts S_t (the renormalised softmax), so
+ *   dz[t][e] = w_e (dw_e - sum_{i in S_t} w_i dw_i)  for e in S_t, else 0;
+ * dlogits = dz (fp32, dense [T][E]); dbias[e] = sum_t dz[t][e] (fp32, may be
+ * NULL).  The selection itself is piecewise constant and passes no gradient. */
+void oracle_route_backward(const int32_t* ids, const float* w, const float* dw, int T, int E,
+                           int k, float* dlogits, float* dbias) {
+    double* db = (double*)calloc((size_t)E, sizeof(double));
+    if (!db) return;
+    for (int t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) dlogits[(int64_t)t * E + e] = 0.0f;
+        double s = 0.0;
+        for (int i = 0; i < k; ++i) s += (double)w[(int64_t)t * k + i] * (double)dw[(int64_t)t * k + i];
+        for (int j = 0; j < k; ++j) {
+            int e = ids[(int64_t)t * k + j];
+            double dz = (double)w[(int64_t)t * k + j] * ((double)dw[(int64_t)t * k + j] - s);
+            dlogits[(int64_t)t * E + e] = (float)dz;
+            db[e] += dz;
+        }
+    }
+    if (dbias)
+        for (int e = 0; e < E; ++e) dbias[e] = (float)db[e];
+    free(db);
+}
+
+/* Gate projection, backward: dx[t][c] += sum_e dlogits[t][e] Wg[e][c] (added
+ * to the dtype values already in dx, rounded once) and
+ * dWg[e][c] = sum_t dlogits[t][e] x[t][c] (fp32). */
+void oracle_gate_backward(const void* x, const void* Wg, int dtype, int T, int d, int E,
+                          const float* dlogits, void* dx, float* dWg) {
+    for (int t = 0; t < T; ++t)
+        for (int c = 0; c < d; ++c) {
+            double acc = load_elem(dx, dtype, (int64_t)t * d + c);
+            for (int e = 0; e < E; ++e)
+                acc += (double)dlogits[(int64_t)t * E + e] * load_elem(Wg, dtype, (int64_t)e * d + c);
+            store_elem(dx, dtype, (int64_t)t * d + c, acc);
+        }
+    for (int e = 0; e < E; ++e)
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int t = 0; t < T; ++t)
+                acc += (double)dlogits[(int64_t)t * E + e] * load_elem(x, dtype, (int64_t)t * d + c);
+            dWg[(int64_t)e * d + c] = (float)acc;
+        }
+}

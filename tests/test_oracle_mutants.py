@@ -32,8 +32,8 @@ MUTANTS = {
     "combine_first_weight_only": ("double wj = (double)w[(int64_t)t * k + j];",
                                   "double wj = (double)w[(int64_t)t * k];"),
     "dispatch_wrong_token": ("int t = row_slot[row] / k;", "int t = row_slot[row] % T;"),
-    "gate_transposed": ("load_elem(Wg, dtype, (int64_t)e * d + c)",
-                        "load_elem(Wg, dtype, (int64_t)c * E + e)"),
+    "gate_transposed": ("*\n                       load_elem(Wg, dtype, (int64_t)e * d + c);",
+                        "*\n                       load_elem(Wg, dtype, (int64_t)c * E + e);"),
     "window_not_clamped": ("int64_t n = step + 1 < W ? step + 1 : W;", "int64_t n = W;"),
     "hot_tie_to_higher": ("if (best < 0 || sum[e] > sum[best]) best = e;",
                           "if (best < 0 || sum[e] >= sum[best]) best = e;"),
@@ -49,6 +49,18 @@ MUTANTS = {
                          "(double)counts[e] / (double)T"),
     "aux_unnormalised_softmax": ("for (int e = 0; e < E; ++e) P[e] += ex[e] / D;",
                                  "for (int e = 0; e < E; ++e) P[e] += ex[e];"),
+    "bwd_no_relu_mask": ("if (load_elem(H, dtype, (int64_t)r * F + f) > 0.0)", "if (1)"),
+    "bwd_w1_transposed": ("acc += g[f] * load_elem(W1, dtype, w1b + (int64_t)f * d + c);",
+                          "acc += g[f] * load_elem(W1, dtype, w1b + (int64_t)c * F + f);"),
+    "bwd_route_no_centering": ("((double)dw[(int64_t)t * k + j] - s)",
+                               "((double)dw[(int64_t)t * k + j])"),
+    "bwd_dispatch_first_slot": ("if (row >= 0) acc += load_elem(dXp",
+                                "if (row >= 0 && j == 0) acc += load_elem(dXp"),
+    "bwd_combine_unweighted": ("store_elem(dYp, dtype, (int64_t)row * d + o, (double)w[s] * g);",
+                               "store_elem(dYp, dtype, (int64_t)row * d + o, g);"),
+    "bwd_gate_wrong_operand": (
+        "acc += (double)dlogits[(int64_t)t * E + e] * load_elem(x, dtype, (int64_t)t * d + c);",
+        "acc += (double)dlogits[(int64_t)t * E + e] * load_elem(Wg, dtype, (int64_t)e * d + c);"),
     "forecast_column_sum": ("a += q[i] * (double)C[(int64_t)i * E + h];",
                             "a += q[i] * (double)C[(int64_t)h * E + i];"),
 }
@@ -66,6 +78,7 @@ def test_pins_reject_mutant(name, tmp_path):
                            "-fPIC", "-shared", "-o", str(lib), str(mutated), "-lm"])
     env = dict(os.environ, MOE_ORACLE_LIB=str(lib))
     res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                          os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                          os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                          os.path.join(ROOT, "tests", "test_oracle_backward.py")],
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert res.returncode != 0, f"pins accepted the mutant {name}:\n{res.stdout[-2000:]}"
