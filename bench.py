@@ -82,7 +82,7 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-GEMM_SOURCES = ["gemm_tc.cu", "grouped.cuh", "common.cuh"]
+GEMM_SOURCES = ["gemm_tc.cu", "tc_ptx.cuh", "grouped.cuh", "common.cuh"]
 
 
 def gemm_traffic(workload: str, kernel: str):
@@ -238,6 +238,70 @@ def reference_arm(args, w):
 
 
 # ------------------------------------------------------------------ ours ---
+def backward_extras(moe, w, layer, b, weights, stream, torch, reps=20):
+    """Times the layer's backward (after a forward of batch b) stage by stage:
+    combine, expert FFN (input gradients alone, then with weight gradients),
+    dispatch, route and gate backward, each with events around it."""
+    dy_np = wl.make_grad(w, 1)
+    dy = (torch.from_numpy(dy_np.view(np.int16)).view(torch.bfloat16)
+          if dy_np.dtype == np.uint16 else torch.from_numpy(dy_np)).cuda()
+    Wg, W1, W2 = weights.get("Wg"), weights.get("W1"), weights.get("W2")
+    layer.forward(b["x"], Wg, W1, W2, b["bias"], logits=b.get("logits"), popularity=False)
+    layer.backward(dy, b["x"], Wg, W1, W2)  # allocates the gradient buffers
+    R = int(layer.offsets[-1].item())
+    names = ["combine_bwd", "ffn_bwd_input", "ffn_bwd_weights", "dispatch_bwd", "route_bwd",
+             "gate_bwd"]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+          for _ in range(reps)]
+    for i in range(reps + 3):
+        e = ev[i - 3] if i >= 3 else None
+        rec = (lambda j: e[j].record(stream)) if e else (lambda j: None)
+        rec(0)
+        moe.moe_combine_backward(dy, layer.Yp, w.k, layer.slot_row, layer.w, layer.dw, layer.dYp)
+        rec(1)
+        if not w.identity_experts:
+            moe.moe_expert_ffn_backward(layer.Xp, layer.H, layer.dYp, W1, W2, layer.offsets,
+                                        layer.dH, layer.dXp, None, None)
+        rec(2)
+        if not w.identity_experts:
+            moe.moe_expert_ffn_backward(layer.Xp, layer.H, layer.dYp, W1, W2, layer.offsets,
+                                        layer.dH, layer.dXp, layer.dW1, layer.dW2)
+        rec(3)
+        moe.moe_dispatch_backward(layer.dXp, w.k, layer.slot_row, layer.dx)
+        rec(4)
+        moe.moe_route_backward(layer.ids, layer.w, layer.dw, w.E, layer.dlogits, layer.dbias,
+                               layer.workspace)
+        rec(5)
+        if Wg is not None:
+            moe.moe_gate_backward(b["x"], Wg, layer.dlogits, layer.dx, layer.dWg)
+        rec(6)
+    torch.cuda.synchronize()
+    ms = np.zeros(len(names))
+    for e in ev:
+        ms += np.array([e[j].elapsed_time(e[j + 1]) for j in range(len(names))])
+    ms /= reps
+    es = 2 if w.dtype == "bf16" else 4
+    out = {n: {"ms": float(m)} for n, m in zip(names, ms)}
+    if not w.identity_experts:
+        # the second call redoes the two input-gradient GEMMs, then the two
+        # weight-gradient GEMMs: its excess over the first is theirs
+        wgt_ms = float(ms[2] - ms[1])
+        out["ffn_bwd_weights"] = {"ms_all_four": float(ms[2]), "ms_weight_gemms": wgt_ms}
+        out["ffn_bwd_input"]["tflops"] = 4.0 * R * w.d * w.F / (ms[1] * 1e-3) / 1e12
+        if wgt_ms > 0:
+            out["ffn_bwd_weights"]["tflops"] = 4.0 * R * w.d * w.F / (wgt_ms * 1e-3) / 1e12
+    out["combine_bwd"]["gbs"] = (R * w.d * es * 2 + w.T * w.d * es) / (ms[0] * 1e-3) / 1e9
+    out["dispatch_bwd"]["gbs"] = (R * w.d * es + w.T * w.d * es) / (ms[3] * 1e-3) / 1e9
+    out["route_bwd"]["gbs"] = w.T * w.E * 4 / (ms[4] * 1e-3) / 1e9
+    if Wg is not None:
+        out["gate_bwd"]["tflops"] = 4.0 * w.T * w.d * w.E / (ms[5] * 1e-3) / 1e12
+    out["step_ms"] = float(ms[0] + ms[2:].sum())
+    out["R"] = R
+    out["note"] = (f"{reps} backward passes after one forward, events around each call; "
+                   "step_ms = combine + FFN (all four GEMMs) + dispatch + route + gate")
+    return out
+
+
 def main():
     args = parse()
     w = workload_of(args)
@@ -460,7 +524,9 @@ def main():
         torch.cuda.synchronize()
         aux_ms = ev[0].elapsed_time(ev[1]) / reps
         corr_bytes = 2 * w.T * w.k * 4 + 2 * w.E * w.E * 4
+        bwd = backward_extras(moe, w, layer, batches[1 % nb], weights, stream, torch)
         extras = {
+            "backward": bwd,
             "correlation_update": {"ms": corr_ms, "pairs": w.T * w.k * w.k,
                                    "gbs": corr_bytes / (corr_ms * 1e-3) / 1e9},
             "popularity_forecast": {"ms": fc_ms, "E": w.E},

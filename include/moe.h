@@ -13,6 +13,9 @@
  *   moe_combine            output decode: gate-weighted un-permute      (a4)
  *   moe_popularity_update  per-expert popularity, sliding-window mean   (a5)
  *
+ * and the backward of each step (moe_combine_backward, moe_expert_ffn_backward,
+ * moe_dispatch_backward, moe_route_backward, moe_gate_backward).
+ *
  * Conventions shared by every call
  *  - All tensor pointers are DEVICE pointers to memory the caller owns.  The
  *    library allocates nothing; the only scratch (moe_route's) is a caller
@@ -260,6 +263,73 @@ MOE_API int moe_popularity_forecast(const float* pop_prev, const int32_t* C, int
 MOE_API int moe_aux_loss(const float* logits, const float* bias, int T, int E, int k,
                          const int32_t* counts, float* loss, float* prob_mean, void* workspace,
                          size_t workspace_bytes, moe_stream_t stream);
+
+/* ------------------------------------------------------------ backward --
+ * Gradients of the layer above.  PopFetcher, section 5.2.1: each expert GEMM
+ * of the forward pass has two in the backward pass, one for its input and one
+ * for its weights.  The other steps are the adjoints of the forward gathers
+ * and of the gate's softmax.  The forward values they need (Yp, H, Xp, w,
+ * ids, slot_row, offsets) are the ones the forward calls wrote.
+ */
+
+/* Output decode, backward.  For every kept slot (row = slot_row[t][j] >= 0):
+ *   dw[t][j] = <dy[t], Yp[row]>     fp32 (lanes in fp32, fixed-order sum)
+ *   dYp[row] = w[t][j] * dy[t]      the exact product rounded once to dtype
+ * and dw[t][j] = 0 for a dropped slot.  dy [T, d], Yp and dYp [R_max, d]
+ * dtype; slot_row, w, dw [T, k].  Rows of dYp no slot names are not written.
+ */
+MOE_API int moe_combine_backward(const void* dy, const void* Yp, int dtype, int T, int d, int k,
+                                 const int32_t* slot_row, const float* w, float* dw, void* dYp,
+                                 int R_max, moe_stream_t stream);
+
+/* Expert computation, backward, for the rows r of each group e
+ * (offsets[e] <= r < offsets[e+1]):
+ *   dH[r][f]     = H[r][f] > 0 ? sum_o dYp[r][o] W2[e][o][f] : 0   (ReLU)
+ *   dXp[r][c]    = sum_f dH[r][f] W1[e][f][c]
+ *   dW2[e][o][f] = sum_r dYp[r][o] H[r][f]
+ *   dW1[e][f][c] = sum_r dH[r][f] Xp[r][c]
+ * dH and dXp [R_max, F] / [R_max, d] in dtype (the stored dH feeds dXp and
+ * dW1); dW1 [E, F, d] and dW2 [E, d, F] fp32, either may be NULL; an expert
+ * with no rows gets zero weight gradients.  Accumulation in fp32: bf16 on the
+ * tcgen05 tensor cores (weights read in their forward layout as N-major
+ * operands), fp32 on the CUDA cores.  Same alignment rules as moe_expert_ffn.
+ */
+MOE_API int moe_expert_ffn_backward(const void* Xp, const void* H, const void* dYp, const void* W1,
+                                    const void* W2, int dtype, int E, int d, int F,
+                                    const int32_t* offsets, int R_max, void* dH, void* dXp,
+                                    float* dW1, float* dW2, moe_stream_t stream);
+
+/* Input encode, backward: dx[t] = sum of dXp[slot_row[t][j]] over the token's
+ * kept slots, j ascending, accumulated in fp32 and rounded once to dtype
+ * (zeros for a token whose slots were all dropped).  dXp [R_max, d], dx [T, d].
+ */
+MOE_API int moe_dispatch_backward(const void* dXp, int dtype, int T, int d, int k,
+                                  const int32_t* slot_row, void* dx, int R_max,
+                                  moe_stream_t stream);
+
+/* Gate routing, backward.  The gate weights are the softmax renormalised over
+ * the token's selected experts S_t, so for e in S_t
+ *   dlogits[t][e] = w_e (dw_e - sum_{i in S_t} w_i dw_i)
+ * taken in double (each operation rounded, i ascending) and rounded to fp32;
+ * dlogits [T, E] fp32 is dense, zero off S_t (the selection passes no
+ * gradient).  dbias [E] fp32 = sum_t dlogits[t][e] (NULL: skipped); it needs
+ * a workspace of moe_route_workspace_size(T, E, k) bytes (the router's may be
+ * reused).  ids, w [T, k] from moe_route; dw [T, k] from moe_combine_backward.
+ * Deterministic.
+ */
+MOE_API int moe_route_backward(const int32_t* ids, const float* w, const float* dw, int T, int E,
+                               int k, float* dlogits, float* dbias, void* workspace,
+                               size_t workspace_bytes, moe_stream_t stream);
+
+/* Gate projection, backward (logits = x . Wg^T):
+ *   dx[t][c] += sum_e dlogits[t][e] Wg[e][c]   added to dx in place, rounded
+ *                                              once to dtype
+ *   dWg[e][c] = sum_t dlogits[t][e] x[t][c]    fp32 (NULL: skipped)
+ * x, dx [T, d] and Wg [E, d] in dtype; dlogits [T, E] fp32.  fp32 products on
+ * the CUDA cores (the router stays fp32 end to end).
+ */
+MOE_API int moe_gate_backward(const void* x, const void* Wg, int dtype, int T, int d, int E,
+                              const float* dlogits, void* dx, float* dWg, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

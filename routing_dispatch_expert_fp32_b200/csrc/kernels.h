@@ -23,4 +23,25 @@ bool gate_small_fits(int E, int d, int dtype);
 int launch_gate_small(const void* x, const void* Wg, int dtype, int T, int d, int E,
                       float* logits, cudaStream_t st);
 
+// Backward of the expert FFN over the grouped rows (gemm_bwd.cu for bf16 on
+// tcgen05, gemm_simt.cu for fp32): dH = (dYp . W2_e) masked by H > 0,
+// dXp = dH . W1_e, and (when non-null) dW2_e = dYp_e^T H_e, dW1_e = dH_e^T Xp_e
+// in fp32.
+int launch_ffn_backward_bf16(const void* Xp, const void* H, const void* dYp, const void* W1,
+                             const void* W2, int E, int d, int F, const int32_t* offsets,
+                             int R_max, void* dH, void* dXp, float* dW1, float* dW2,
+                             cudaStream_t st);
+int launch_ffn_backward_f32(const float* Xp, const float* H, const float* dYp, const float* W1,
+                            const float* W2, int E, int d, int F, const int32_t* offsets,
+                            int R_max, float* dH, float* dXp, float* dW1, float* dW2,
+                            cudaStream_t st);
+
+// Epilogues of the CUDA-core backward product (gemm_simt.cu).
+enum { SIMT_EPI_STORE = 0, SIMT_EPI_MASK = 1, SIMT_EPI_ADD = 2 };
+
+// Gate projection backward on the CUDA cores (gemm_simt.cu):
+// dx += dlogits . Wg, and dWg = dlogits^T . x (fp32) when dWg is non-null.
+int launch_gate_backward(const void* x, const void* Wg, int dtype, int T, int d, int E,
+                         const float* dlogits, void* dx, float* dWg, cudaStream_t st);
+
 }  // namespace moe

@@ -6,6 +6,9 @@
 // indices (here with the gate weights applied, as the layer output is the
 // gate-weighted sum of the selected experts' outputs).
 //
+// The backward of input encode (moe_dispatch_backward) is the same gather as
+// output decode with unit weights: dx[t] = sum of the token's kept rows of dXp.
+//
 // Both are HBM-bound row copies.  Token-parallel: one warp owns one token row
 // at a time (grid-stride over tokens), moves it in 16-byte vectors with
 // U vectors per lane in flight, and
@@ -109,7 +112,7 @@ combine_kernel(const uint4* __restrict__ Yp, int T, int nvec, int k,
         float my_w = 0.0f;
         if (lane < k) {
             my_row = __ldg(slot_row + (size_t)t * k + lane);
-            my_w = __ldg(w + (size_t)t * k + lane);
+            my_w = w ? __ldg(w + (size_t)t * k + lane) : 1.0f;
             if (my_row < -1 || my_row >= R_max) {
                 flag_error(err, MOE_DEVERR_ROW_INDEX);
                 my_row = -1;
@@ -190,4 +193,20 @@ extern "C" MOE_API int moe_combine(const void* Yp, int dtype, int T, int d, int 
                                         : combine_kernel<MOE_DTYPE_F32>;
     return launch_pdl(kern, perm_grid(T), kPermThreads, 0, st, static_cast<const uint4*>(Yp), T,
                       nvec, k, slot_row, w, static_cast<uint4*>(y), R_max, device_error_word());
+}
+
+extern "C" MOE_API int moe_dispatch_backward(const void* dXp, int dtype, int T, int d, int k,
+                                             const int32_t* slot_row, void* dx, int R_max,
+                                             moe_stream_t stream) {
+    const int rc = check_rows(dXp, dx, dtype, T, d, k);
+    if (rc != MOE_OK) return rc;
+    if (T > 0 && (!slot_row || R_max < 0)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    const int nvec = (int)((size_t)d * dtype_bytes(dtype) / 16);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    auto kern = dtype == MOE_DTYPE_BF16 ? combine_kernel<MOE_DTYPE_BF16>
+                                        : combine_kernel<MOE_DTYPE_F32>;
+    return launch_pdl(kern, perm_grid(T), kPermThreads, 0, st, static_cast<const uint4*>(dXp), T,
+                      nvec, k, slot_row, static_cast<const float*>(nullptr), static_cast<uint4*>(dx),
+                      R_max, device_error_word());
 }

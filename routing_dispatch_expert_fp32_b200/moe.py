@@ -44,6 +44,12 @@ _SIGS = {
     "moe_correlation_update": ([_p, _i, _p, _i, _i, _i, _p, _p], _i),
     "moe_popularity_forecast": ([_p, _p, _i, _i, _i, _p, _i, _p, _p], _i),
     "moe_aux_loss": ([_p, _p, _i, _i, _i, _p, _p, _p, _p, _sz, _p], _i),
+    "moe_combine_backward": ([_p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p], _i),
+    "moe_expert_ffn_backward": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _p, _p, _p, _p],
+                                _i),
+    "moe_dispatch_backward": ([_p, _i, _i, _i, _i, _p, _p, _i, _p], _i),
+    "moe_route_backward": ([_p, _p, _p, _i, _i, _i, _p, _p, _p, _sz, _p], _i),
+    "moe_gate_backward": ([_p, _p, _i, _i, _i, _i, _p, _p, _p, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -171,6 +177,43 @@ def moe_aux_loss(logits, bias, k, counts, loss, prob_mean, workspace, stream=Non
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def moe_combine_backward(dy, Yp, k, slot_row, w, dw, dYp, stream=None):
+    T, d = dy.shape
+    _check("moe_combine_backward", lib.moe_combine_backward(
+        _ptr(dy), _ptr(Yp), dtype_code(dy), T, d, k, _ptr(slot_row), _ptr(w), _ptr(dw),
+        _ptr(dYp), Yp.shape[0], _stream(stream)))
+
+
+def moe_expert_ffn_backward(Xp, H, dYp, W1, W2, offsets, dH, dXp, dW1, dW2, stream=None):
+    E, F, d = W1.shape
+    _check("moe_expert_ffn_backward", lib.moe_expert_ffn_backward(
+        _ptr(Xp), _ptr(H), _ptr(dYp), _ptr(W1), _ptr(W2), dtype_code(Xp), E, d, F,
+        _ptr(offsets), Xp.shape[0], _ptr(dH), _ptr(dXp), _ptr(dW1), _ptr(dW2), _stream(stream)))
+
+
+def moe_dispatch_backward(dXp, k, slot_row, dx, stream=None):
+    T, d = dx.shape
+    _check("moe_dispatch_backward", lib.moe_dispatch_backward(
+        _ptr(dXp), dtype_code(dXp), T, d, k, _ptr(slot_row), _ptr(dx), dXp.shape[0],
+        _stream(stream)))
+
+
+def moe_route_backward(ids, w, dw, E, dlogits, dbias, workspace, stream=None):
+    T, k = ids.shape
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("moe_route_backward", lib.moe_route_backward(
+        _ptr(ids), _ptr(w), _ptr(dw), T, E, k, _ptr(dlogits), _ptr(dbias), _ptr(workspace),
+        nbytes, _stream(stream)))
+
+
+def moe_gate_backward(x, Wg, dlogits, dx, dWg, stream=None):
+    T, d = x.shape
+    E = Wg.shape[0]
+    _check("moe_gate_backward", lib.moe_gate_backward(
+        _ptr(x), _ptr(Wg), dtype_code(x), T, d, E, _ptr(dlogits), _ptr(dx), _ptr(dWg),
+        _stream(stream)))
+
+
 class MoELayer:
     """One MoE layer's device buffers plus the call sequence of the hot path.
 
@@ -226,6 +269,59 @@ class MoELayer:
             moe_expert_ffn(self.Xp, W1, W2, self.offsets, self.H, self.Yp, stream)
         moe_combine(self.Yp, self.k, self.slot_row, self.w, self.y, stream)
         return self.y
+
+    def backward(self, dy, x, Wg=None, W1=None, W2=None, stream=None, weight_grads=True):
+        """Gradients of the last ``forward`` given dy = dLoss/dy.
+
+        Runs combine, expert-FFN, dispatch, route and gate backward through the
+        C ABI on the forward's stored tensors and returns a dict with dx,
+        dlogits, dbias and (when ``weight_grads``) dW1, dW2, dWg; dWg and the
+        gate's share of dx only when Wg is given (the forward ran the gate).
+        """
+        T, d, E, k, F = self.T, self.d, self.E, self.k, self.F
+        dev = self.y.device
+        if not hasattr(self, "dYp"):
+            Rmax = self.Xp.shape[0]
+            self.dw = torch.empty(T, k, dtype=torch.float32, device=dev)
+            self.dYp = torch.empty(Rmax, d, dtype=self.dtype, device=dev)
+            self.dH = None if self.identity_experts else torch.empty(Rmax, F, dtype=self.dtype,
+                                                                     device=dev)
+            self.dXp = self.dYp if self.identity_experts else torch.empty(
+                Rmax, d, dtype=self.dtype, device=dev)
+            self.dx = torch.empty(T, d, dtype=self.dtype, device=dev)
+            self.dlogits = torch.empty(T, E, dtype=torch.float32, device=dev)
+            self.dbias = torch.empty(E, dtype=torch.float32, device=dev)
+            self.dW1 = None if self.identity_experts else torch.empty(E, F, d, dtype=torch.float32,
+                                                                      device=dev)
+            self.dW2 = None if self.identity_experts else torch.empty(E, d, F, dtype=torch.float32,
+                                                                      device=dev)
+            self.dWg = torch.empty(E, d, dtype=torch.float32, device=dev)
+        moe_combine_backward(dy, self.Yp, k, self.slot_row, self.w, self.dw, self.dYp, stream)
+        if not self.identity_experts:
+            moe_expert_ffn_backward(self.Xp, self.H, self.dYp, W1, W2, self.offsets, self.dH,
+                                    self.dXp, self.dW1 if weight_grads else None,
+                                    self.dW2 if weight_grads else None, stream)
+        moe_dispatch_backward(self.dXp, k, self.slot_row, self.dx, stream)
+        moe_route_backward(self.ids, self.w, self.dw, E, self.dlogits, self.dbias,
+                           self.workspace, stream)
+        out = dict(dx=self.dx, dlogits=self.dlogits, dbias=self.dbias)
+        if Wg is not None:
+            moe_gate_backward(x, Wg, self.dlogits, self.dx,
+                              self.dWg if weight_grads else None, stream)
+            if weight_grads:
+                out["dWg"] = self.dWg
+        if weight_grads and not self.identity_experts:
+            out.update(dW1=self.dW1, dW2=self.dW2)
+        return out
+
+    def launches_per_backward(self, gate=True, weight_grads=True) -> int:
+        """Kernel launches one backward makes."""
+        n = 1 + 1 + 2  # combine, dispatch, route (dlogits + dbias)
+        if not self.identity_experts:
+            n += 4 if weight_grads else 2
+        if gate:
+            n += 2 if weight_grads else 1
+        return n
 
     def capture(self, x, Wg=None, W1=None, W2=None, bias=None, logits=None, popularity=True):
         """Records one ``forward`` on these tensors into a CUDA graph and returns it.

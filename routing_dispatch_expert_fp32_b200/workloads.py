@@ -29,6 +29,7 @@ from fractions import Fraction
 import numpy as np
 
 TENSOR_X, TENSOR_WG, TENSOR_W1, TENSOR_W2, TENSOR_BIAS, TENSOR_LOGITS, TENSOR_PERM = range(7)
+TENSOR_DY, TENSOR_XP, TENSOR_H, TENSOR_DYP = range(7, 11)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -156,6 +157,26 @@ def make_step(w: Workload, step: int = 0, rank: int = 0) -> dict:
         out["logits"] = rng_for(w, step, TENSOR_LOGITS, rank).standard_normal(
             (w.T, w.E), dtype=np.float32)
     return out
+
+
+def make_grad(w: Workload, step: int = 0, rank: int = 0) -> np.ndarray:
+    """Upstream gradient of the layer output, dy ~ N(0, 1) [T, d] in the layer's dtype."""
+    return _normal(rng_for(w, step, TENSOR_DY, rank), (w.T, w.d), 1.0, w.dtype)
+
+
+def router_logits(w: Workload, step: int = 0, rank: int = 0) -> np.ndarray:
+    """Router scores ~ N(0, 1) [T, E] fp32 (the workload's bias adds its skew)."""
+    return rng_for(w, step, TENSOR_LOGITS, rank).standard_normal((w.T, w.E), dtype=np.float32)
+
+
+def ffn_backward_inputs(w: Workload, R_max: int, step: int = 0, rank: int = 0) -> dict:
+    """Grouped rows for the expert backward alone: Xp, dYp ~ N(0, 1) [R_max, d] and
+    H = max(0, N(0, 1)) [R_max, F] (about half exact zeros, as after a ReLU)."""
+    H = rng_for(w, step, TENSOR_H, rank).standard_normal((R_max, w.F), dtype=np.float32)
+    np.maximum(H, 0.0, out=H)
+    return {"Xp": _normal(rng_for(w, step, TENSOR_XP, rank), (R_max, w.d), 1.0, w.dtype),
+            "H": to_bf16_bits(H) if w.dtype == "bf16" else H,
+            "dYp": _normal(rng_for(w, step, TENSOR_DYP, rank), (R_max, w.d), 1.0, w.dtype)}
 
 
 def tiny(name: str, T: int, d: int, E: int, k: int, F: int, dtype: str = "bf16",

@@ -73,7 +73,8 @@ def check_layer(moe, w: wl.Workload, step_inputs, weights, layer, rng, n_tokens=
     rows = sample_rows(r["offsets"], None, rng)
     expert_of_row = np.searchsorted(r["offsets"], rows, side="right") - 1
     rows_d = torch.from_numpy(rows).cuda()
-    Yr, Hr = oracle.expert_ffn_rows(host(layer.Xp[rows_d]), expert_of_row, weights["W1"],
+    # the rows' inputs are their tokens' x (the dispatch check above)
+    Yr, Hr = oracle.expert_ffn_rows(x[r["row_slot"][rows] // w.k], expert_of_row, weights["W1"],
                                     weights["W2"], want_h=True)
     assert_close(host(layer.H[rows_d]), Hr, "H rows")
     assert_close(host(layer.Yp[rows_d]), Yr, "Yp rows")
