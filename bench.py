@@ -273,7 +273,7 @@ def backward_extras(moe, w, layer, b, weights, stream, torch, reps=20):
                                layer.workspace)
         rec(5)
         if Wg is not None:
-            moe.moe_gate_backward(b["x"], Wg, layer.dlogits, layer.dx, layer.dWg)
+            moe.moe_gate_backward(b["x"], Wg, layer.dlogits, layer.dx, layer.dWg, layer.gate_ws)
         rec(6)
     torch.cuda.synchronize()
     ms = np.zeros(len(names))

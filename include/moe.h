@@ -325,11 +325,22 @@ MOE_API int moe_route_backward(const int32_t* ids, const float* w, const float* 
  *   dx[t][c] += sum_e dlogits[t][e] Wg[e][c]   added to dx in place, rounded
  *                                              once to dtype
  *   dWg[e][c] = sum_t dlogits[t][e] x[t][c]    fp32 (NULL: skipped)
- * x, dx [T, d] and Wg [E, d] in dtype; dlogits [T, E] fp32.  fp32 products on
- * the CUDA cores (the router stays fp32 end to end).
+ * x, dx [T, d] and Wg [E, d] in dtype; dlogits [T, E] fp32, and the router
+ * gradient keeps its fp32 precision on both paths:
+ *  - bf16 with d and E multiples of 8: tcgen05 tensor cores; dlogits is split
+ *    exactly into three bf16 planes (hi + mid + lo = dlogits), so every
+ *    product with the bf16 x or Wg is exact and accumulates in fp32;
+ *  - otherwise fp32 products on the CUDA cores.
+ * dWg sums the tokens in consecutive slices whose fp32 partial products are
+ * then added in slice order; the slicing depends on (T, d, E) only, so the
+ * result is the same on every run and every device.  workspace: at least
+ * moe_gate_backward_workspace_size(T, d, E, dtype) bytes (0: NULL accepted).
  */
+MOE_API size_t moe_gate_backward_workspace_size(int T, int d, int E, int dtype);
+
 MOE_API int moe_gate_backward(const void* x, const void* Wg, int dtype, int T, int d, int E,
-                              const float* dlogits, void* dx, float* dWg, moe_stream_t stream);
+                              const float* dlogits, void* dx, float* dWg, void* workspace,
+                              size_t workspace_bytes, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

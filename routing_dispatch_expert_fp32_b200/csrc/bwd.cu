@@ -10,12 +10,13 @@
 //   dYp[row] = w[t][j] * dy[t] (the product taken exactly in double and
 //   rounded once to the row's type).  HBM-bound: dy is read once per slot
 //   (k times, from L1/L2 after the first), Yp read and dYp written once.
-// moe_route_backward: one warp per token; the renormalised softmax over the
+// moe_route_backward: a lane per token; the renormalised softmax over the
 //   token's selected experts gives dz_j = w_j (dw_j - sum_i w_i dw_i), taken
 //   in double with every operation rounded separately and i ascending, then
 //   rounded once to fp32; dlogits is dense [T][E] (zero off the selection).
-//   dbias = column sums of dlogits: per 256-token chunk in double (tokens
-//   ascending), then over chunks ascending -- deterministic.
+//   dbias = column sums of dlogits: per 256-token chunk in double (fixed
+//   slices of tokens, then the slices), then over chunks ascending --
+//   deterministic.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -117,46 +118,87 @@ combine_backward_kernel(const uint4* __restrict__ dy, const uint4* __restrict__ 
     }
 }
 
-// dlogits rows of one chunk of tokens, then (when dbias is wanted) the chunk's
-// column sums in double.
+// dlogits rows of one chunk of 256 tokens, then (when dbias is wanted) the
+// chunk's column sums in double.  Each warp takes 32 consecutive tokens at
+// once, a lane per token (the loads of all 32 tokens are in flight together):
+// the warp zeroes the 32 rows (one contiguous block of 32*E floats), then each
+// lane writes its token's k entries.  Column sums: S = 256 / E slices of the
+// chunk's tokens per expert (E <= 256), each summed by one thread in token
+// order, then the slices in order -- a fixed order for a given E.
 __global__ void __launch_bounds__(kBwdThreads)
 route_backward_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w,
                       const float* __restrict__ dw, int T, int E, int k,
                       float* __restrict__ dlogits, double* __restrict__ partial, int32_t* err) {
+    __shared__ double s_part[kBwdThreads];
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int kWarps = kBwdThreads / 32;
     const int t0 = blockIdx.x * kBwdChunk;
     const int t1 = min(T, t0 + kBwdChunk);
-    for (int t = t0 + warp; t < t1; t += kWarps) {
-        float* row = dlogits + (size_t)t * E;
-        for (int e = lane; e < E; e += 32) row[e] = 0.0f;
-        __syncwarp();
-        // s = sum_i w_i dw_i, i ascending, each product and sum rounded in double
-        double s = 0.0;
-        for (int i = 0; i < k; ++i) {
-            const double wi = (double)__ldg(w + (size_t)t * k + i);
-            const double gi = (double)__ldg(dw + (size_t)t * k + i);
-            s = __dadd_rn(s, __dmul_rn(wi, gi));
+    const int tw = t0 + warp * 32;  // this warp's first token
+    if (tw < t1) {
+        const int nt = min(32, t1 - tw);
+        // zero rows [tw, tw + nt): contiguous, 16-byte vectors where aligned
+        float* blk = dlogits + (size_t)tw * E;
+        const size_t n = (size_t)nt * E;
+        if ((reinterpret_cast<uintptr_t>(blk) & 15u) == 0) {
+            const size_t nv = n / 4;
+            for (size_t i = lane; i < nv; i += 32)
+                reinterpret_cast<float4*>(blk)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (size_t i = nv * 4 + lane; i < n; i += 32) blk[i] = 0.0f;
+        } else {
+            for (size_t i = lane; i < n; i += 32) blk[i] = 0.0f;
         }
-        for (int j = lane; j < k; j += 32) {
-            const int e = __ldg(ids + (size_t)t * k + j);
-            if (e < 0 || e >= E) {
-                flag_error(err, MOE_DEVERR_EXPERT_INDEX);
-                continue;
+        __syncwarp();
+        const int t = tw + lane;
+        if (lane < nt) {
+            // s = sum_i w_i dw_i, i ascending, each product and sum rounded in double
+            const float* wt = w + (size_t)t * k;
+            const float* gt = dw + (size_t)t * k;
+            double s = 0.0;
+            for (int i = 0; i < k; ++i)
+                s = __dadd_rn(s, __dmul_rn((double)__ldg(wt + i), (double)__ldg(gt + i)));
+            float* row = dlogits + (size_t)t * E;
+            for (int j = 0; j < k; ++j) {
+                const int e = __ldg(ids + (size_t)t * k + j);
+                if (e < 0 || e >= E) {
+                    flag_error(err, MOE_DEVERR_EXPERT_INDEX);
+                    continue;
+                }
+                const double wj = (double)__ldg(wt + j), gj = (double)__ldg(gt + j);
+                row[e] = __double2float_rn(__dmul_rn(wj, __dsub_rn(gj, s)));
             }
-            const double wj = (double)__ldg(w + (size_t)t * k + j);
-            const double gj = (double)__ldg(dw + (size_t)t * k + j);
-            row[e] = __double2float_rn(__dmul_rn(wj, __dsub_rn(gj, s)));
         }
     }
     if (!partial) return;
     __syncthreads();  // the chunk's rows are written (block-scope visibility)
-    for (int e = threadIdx.x; e < E; e += kBwdThreads) {
+    const int n_tok = t1 - t0;
+    if (E <= kBwdThreads) {
+        const int S = kBwdThreads / E;            // slices per expert
+        const int per = (kBwdChunk + S - 1) / S;  // tokens per slice
+        const int e = threadIdx.x % E, sl = threadIdx.x / E;
         double acc = 0.0;
-        for (int t = t0; t < t1; ++t) acc = __dadd_rn(acc, (double)dlogits[(size_t)t * E + e]);
-        partial[(size_t)blockIdx.x * E + e] = acc;
+        if (sl < S) {
+            const int a = sl * per, b = min(n_tok, a + per);
+#pragma unroll 4
+            for (int t = a; t < b; ++t)
+                acc = __dadd_rn(acc, (double)dlogits[(size_t)(t0 + t) * E + e]);
+        }
+        s_part[threadIdx.x] = acc;
+        __syncthreads();
+        if (threadIdx.x < E) {
+            double v = 0.0;
+            for (int q = 0; q < S; ++q) v = __dadd_rn(v, s_part[q * E + threadIdx.x]);
+            partial[(size_t)blockIdx.x * E + threadIdx.x] = v;
+        }
+    } else {
+        for (int e = threadIdx.x; e < E; e += kBwdThreads) {
+            double acc = 0.0;
+#pragma unroll 4
+            for (int t = 0; t < n_tok; ++t)
+                acc = __dadd_rn(acc, (double)dlogits[(size_t)(t0 + t) * E + e]);
+            partial[(size_t)blockIdx.x * E + e] = acc;
+        }
     }
 }
 
@@ -251,12 +293,23 @@ extern "C" MOE_API int moe_route_backward(const int32_t* ids, const float* w, co
                       static_cast<const double*>(partial), nchunks, E, dbias);
 }
 
+extern "C" MOE_API size_t moe_gate_backward_workspace_size(int T, int d, int E, int dtype) {
+    if (T < 0 || d < 1 || E < 1 || !dtype_ok(dtype)) return 0;
+    if (T == 0) return 0;
+    if (dtype == MOE_DTYPE_BF16 && gate_backward_tc_ok(d, E))
+        return gate_backward_tc_workspace(T, d, E);
+    const int ks = gate_backward_splits(T, d, E);
+    return ks > 1 ? (size_t)ks * E * d * sizeof(float) + 256 : 0;
+}
+
 extern "C" MOE_API int moe_gate_backward(const void* x, const void* Wg, int dtype, int T, int d,
                                          int E, const float* dlogits, void* dx, float* dWg,
+                                         void* workspace, size_t workspace_bytes,
                                          moe_stream_t stream) {
     if (!dtype_ok(dtype)) return MOE_ERR_UNSUPPORTED;
     if (T < 0 || d < 1 || E < 1 || E > kMaxExperts) return MOE_ERR_INVALID_ARG;
     if ((int64_t)T * d >= INT32_MAX || (int64_t)T * E >= INT32_MAX) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)T * 3 >= INT32_MAX) return MOE_ERR_INVALID_ARG;
     if (!Wg || (T > 0 && (!x || !dlogits || !dx))) return MOE_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (T == 0) {  // no tokens: dWg = 0
@@ -265,5 +318,17 @@ extern "C" MOE_API int moe_gate_backward(const void* x, const void* Wg, int dtyp
                    ? MOE_OK
                    : MOE_ERR_CUDA;
     }
-    return launch_gate_backward(x, Wg, dtype, T, d, E, dlogits, dx, dWg, st);
+    const size_t need = moe_gate_backward_workspace_size(T, d, E, dtype);
+    if (dtype == MOE_DTYPE_BF16 && gate_backward_tc_ok(d, E)) {
+        if (!workspace || workspace_bytes < need) return MOE_ERR_WORKSPACE;
+        if (!aligned16(x) || !aligned16(Wg) || !aligned16(dx) || !aligned16(dWg))
+            return MOE_ERR_UNSUPPORTED;
+        return launch_gate_backward_bf16(x, Wg, T, d, E, dlogits, dx, dWg, workspace, st);
+    }
+    const size_t need_simt = dWg ? need : 0;
+    if (need_simt && (!workspace || workspace_bytes < need_simt)) return MOE_ERR_WORKSPACE;
+    float* part = need_simt ? reinterpret_cast<float*>(
+                                  (reinterpret_cast<uintptr_t>(workspace) + 255u) & ~uintptr_t(255u))
+                            : nullptr;
+    return launch_gate_backward(x, Wg, dtype, T, d, E, dlogits, dx, dWg, part, st);
 }

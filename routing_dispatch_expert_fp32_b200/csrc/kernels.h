@@ -40,8 +40,26 @@ int launch_ffn_backward_f32(const float* Xp, const float* H, const float* dYp, c
 enum { SIMT_EPI_STORE = 0, SIMT_EPI_MASK = 1, SIMT_EPI_ADD = 2 };
 
 // Gate projection backward on the CUDA cores (gemm_simt.cu):
-// dx += dlogits . Wg, and dWg = dlogits^T . x (fp32) when dWg is non-null.
+// dx += dlogits . Wg, and dWg = dlogits^T . x (fp32) when dWg is non-null,
+// the tokens cut into gate_backward_splits(T, d, E) slices whose partial
+// products go to `part` ([splits][E][d] fp32, unused with one slice).
+int gate_backward_splits(int T, int d, int E);
 int launch_gate_backward(const void* x, const void* Wg, int dtype, int T, int d, int E,
-                         const float* dlogits, void* dx, float* dWg, cudaStream_t st);
+                         const float* dlogits, void* dx, float* dWg, float* part,
+                         cudaStream_t st);
+
+// out[i] = sum over s ascending of part[s * n + i] (gemm_simt.cu).
+int launch_split_reduce(const float* part, int ksplit, size_t n, float* out, cudaStream_t st);
+
+// Gate projection backward of bf16 layers on tcgen05 (gemm_bwd.cu): dlogits
+// split exactly into three bf16 planes; dx += dlogits . Wg, dWg (fp32, when
+// non-null) over token slices added in order.  Needs d and E multiples of 8
+// (gate_backward_tc_ok) and gate_backward_tc_workspace(T, d, E) bytes.
+bool gate_backward_tc_ok(int d, int E);
+void gate_backward_tc_slices(int T, int d, int E, int* S, int* slice_rows);
+size_t gate_backward_tc_workspace(int T, int d, int E);
+int launch_gate_backward_bf16(const void* x, const void* Wg, int T, int d, int E,
+                              const float* dlogits, void* dx, float* dWg, void* ws,
+                              cudaStream_t st);
 
 }  // namespace moe

@@ -49,7 +49,8 @@ _SIGS = {
                                 _i),
     "moe_dispatch_backward": ([_p, _i, _i, _i, _i, _p, _p, _i, _p], _i),
     "moe_route_backward": ([_p, _p, _p, _i, _i, _i, _p, _p, _p, _sz, _p], _i),
-    "moe_gate_backward": ([_p, _p, _i, _i, _i, _i, _p, _p, _p, _p], _i),
+    "moe_gate_backward_workspace_size": ([_i, _i, _i, _i], _sz),
+    "moe_gate_backward": ([_p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _sz, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -206,12 +207,18 @@ def moe_route_backward(ids, w, dw, E, dlogits, dbias, workspace, stream=None):
         nbytes, _stream(stream)))
 
 
-def moe_gate_backward(x, Wg, dlogits, dx, dWg, stream=None):
+def moe_gate_backward_workspace_size(T: int, d: int, E: int, dtype=torch.bfloat16) -> int:
+    code = MOE_DTYPE_BF16 if dtype == torch.bfloat16 else MOE_DTYPE_F32
+    return int(lib.moe_gate_backward_workspace_size(T, d, E, code))
+
+
+def moe_gate_backward(x, Wg, dlogits, dx, dWg, workspace=None, stream=None):
     T, d = x.shape
     E = Wg.shape[0]
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("moe_gate_backward", lib.moe_gate_backward(
         _ptr(x), _ptr(Wg), dtype_code(x), T, d, E, _ptr(dlogits), _ptr(dx), _ptr(dWg),
-        _stream(stream)))
+        _ptr(workspace), nbytes, _stream(stream)))
 
 
 class MoELayer:
@@ -296,6 +303,9 @@ class MoELayer:
             self.dW2 = None if self.identity_experts else torch.empty(E, d, F, dtype=torch.float32,
                                                                       device=dev)
             self.dWg = torch.empty(E, d, dtype=torch.float32, device=dev)
+            self.gate_ws = torch.empty(
+                max(moe_gate_backward_workspace_size(T, d, E, self.dtype), 1), dtype=torch.uint8,
+                device=dev)
         moe_combine_backward(dy, self.Yp, k, self.slot_row, self.w, self.dw, self.dYp, stream)
         if not self.identity_experts:
             moe_expert_ffn_backward(self.Xp, self.H, self.dYp, W1, W2, self.offsets, self.dH,
@@ -307,7 +317,7 @@ class MoELayer:
         out = dict(dx=self.dx, dlogits=self.dlogits, dbias=self.dbias)
         if Wg is not None:
             moe_gate_backward(x, Wg, self.dlogits, self.dx,
-                              self.dWg if weight_grads else None, stream)
+                              self.dWg if weight_grads else None, self.gate_ws, stream)
             if weight_grads:
                 out["dWg"] = self.dWg
         if weight_grads and not self.identity_experts:
@@ -320,7 +330,20 @@ class MoELayer:
         if not self.identity_experts:
             n += 4 if weight_grads else 2
         if gate:
-            n += 2 if weight_grads else 1
+            tc = self.dtype == torch.bfloat16 and self.d % 8 == 0 and self.E % 8 == 0
+            if tc:  # plane split, dx GEMM, dWg GEMM (+ slice reduction)
+                n += 2
+                if weight_grads:
+                    # the workspace holds slice partials beyond the 3 bf16 planes
+                    # (6 T E bytes, rounded up to 256, + 256) only when sliced
+                    planes = (6 * self.T * self.E + 255) // 256 * 256 + 256
+                    n += 2 if lib.moe_gate_backward_workspace_size(
+                        self.T, self.d, self.E, MOE_DTYPE_BF16) > planes else 1
+            else:
+                n += 1
+                if weight_grads:
+                    n += 2 if moe_gate_backward_workspace_size(self.T, self.d, self.E,
+                                                               self.dtype) else 1
         return n
 
     def capture(self, x, Wg=None, W1=None, W2=None, bias=None, logits=None, popularity=True):

@@ -214,7 +214,9 @@ def test_route_backward(moe, T, E, k, cap):
 
 # ---------------------------------------------------------------- gate -----
 @pytest.mark.parametrize("T,d,E,dtype", [(300, 200, 8, "bf16"), (513, 64, 256, "bf16"),
-                                         (100, 136, 16, "f32"), (5, 8, 3, "f32")])
+                                         (100, 136, 16, "f32"), (5, 8, 3, "f32"),
+                                         (4097, 1024, 16, "bf16"), (2000, 72, 1000, "f32"),
+                                         (300, 64, 12, "bf16"), (70, 2056, 64, "bf16")])
 def test_gate_backward(moe, T, d, E, dtype):
     x = rand((T, d), 1.0, dtype, 31)
     Wg = rand((E, d), d ** -0.5, dtype, 32)
@@ -224,7 +226,9 @@ def test_gate_backward(moe, T, d, E, dtype):
     dx_r, dWg_r = oracle.gate_backward(x, Wg, dl, dx0)
     dx = dev(dx0)
     dWg = torch.full((E, d), 4.0, device="cuda")
-    moe.moe_gate_backward(dev(x), dev(Wg), dev(dl), dx, dWg)
+    ws = torch.empty(max(moe.moe_gate_backward_workspace_size(T, d, E, tdt(dtype)), 1),
+                     dtype=torch.uint8, device="cuda")
+    moe.moe_gate_backward(dev(x), dev(Wg), dev(dl), dx, dWg, ws)
     torch.cuda.synchronize()
     tol = dict(max_abs_frac=1e-5, mean_rel=1e-6) if dtype == "f32" else {}
     assert_close(host(dx), dx_r, "dx", **tol)
