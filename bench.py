@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--experts", type=int, default=0,
                     help="override E (smaller profiling cases of the same shapes)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="unfused", choices=["unfused", "fused"],
+                    help="fused: gather the first GEMM's rows from x and weight the second "
+                         "GEMM's rows (no dispatch pass); bf16 expert layers only")
     ap.add_argument("--no-graph", action="store_true",
                     help="issue the step kernel by kernel instead of replaying a CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -107,7 +110,7 @@ def gemm_traffic(workload: str, kernel: str):
     return None
 
 
-def config_of(w: wl.Workload, n: int):
+def config_of(w: wl.Workload, n: int, fused: bool = False):
     c = {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "F": w.F,
          "capacity": w.capacity, "zipf_s": w.zipf_s, "global_batch_tokens": w.T * n,
          "parallelism": f"dp{n}" if n > 1 else "single",
@@ -118,6 +121,7 @@ def config_of(w: wl.Workload, n: int):
         c["experts"] = "identity"
     if w.steps > 1:
         c["popularity_window"] = w.W
+    c["path"] = "fused" if fused else "unfused"
     return c
 
 
@@ -334,7 +338,7 @@ def main():
         inp = wl.make_step(w, s, rank)
         batches.append({k: (None if v is None else to_dev(v)) for k, v in inp.items()})
     layer = moe.MoELayer(w.T, w.d, w.E, w.k, w.F, tdt, capacity=w.capacity, W=w.W, P=w.P,
-                         identity_experts=w.identity_experts)
+                         identity_experts=w.identity_experts, fused=args.path == "fused")
     stream = torch.cuda.current_stream()
     hook = None
     if world > 1:
@@ -362,13 +366,17 @@ def main():
         moe.moe_popularity_update_dev(layer.counts, layer.hist, layer.step_dev, layer.mean,
                                       layer.P, layer.hot)
         ev[2].record(stream)
-        moe.moe_dispatch(b["x"], w.k, layer.slot_row, layer.Xp)
+        if not layer.fused:
+            moe.moe_dispatch(b["x"], w.k, layer.slot_row, layer.Xp)
         ev[3].record(stream)
-        if not w.identity_experts:
+        if layer.fused:
+            moe.moe_expert_ffn_gather(b["x"], w.k, layer.row_slot, layer.w, weights["W1"],
+                                      weights["W2"], layer.offsets, layer.H, layer.Yp)
+        elif not w.identity_experts:
             moe.moe_expert_ffn(layer.Xp, weights["W1"], weights["W2"], layer.offsets, layer.H,
                                layer.Yp)
         ev[4].record(stream)
-        moe.moe_combine(layer.Yp, w.k, layer.slot_row, layer.w, layer.y)
+        moe.moe_combine(layer.Yp, w.k, layer.slot_row, None if layer.fused else layer.w, layer.y)
         ev[5].record(stream)
 
     # R per batch (untimed): algorithmic work of each step
@@ -524,7 +532,8 @@ def main():
         torch.cuda.synchronize()
         aux_ms = ev[0].elapsed_time(ev[1]) / reps
         corr_bytes = 2 * w.T * w.k * 4 + 2 * w.E * w.E * 4
-        bwd = backward_extras(moe, w, layer, batches[1 % nb], weights, stream, torch)
+        bwd = (None if layer.fused else
+               backward_extras(moe, w, layer, batches[1 % nb], weights, stream, torch))
         extras = {
             "backward": bwd,
             "correlation_update": {"ms": corr_ms, "pairs": w.T * w.k * w.k,
@@ -545,7 +554,8 @@ def main():
         alg = {
             "gate": (2.0 * w.T * w.d * w.E, "flop") if not w.logits_direct else (0, "flop"),
             "route+popularity": (w.T * w.E * 4 + w.T * w.k * 4 * 4 + R_mean * 4, "byte"),
-            "dispatch": (w.T * w.d * es + R_mean * w.d * es + w.T * w.k * 4, "byte"),
+            "dispatch": ((0 if layer.fused else w.T * w.d * es + R_mean * w.d * es
+                          + w.T * w.k * 4), "byte"),
             "expert_ffn": (4.0 * R_mean * w.d * w.F, "flop"),
             "combine": (R_mean * w.d * es + w.T * w.d * es + w.T * w.k * 8, "byte"),
         }
@@ -571,7 +581,7 @@ def main():
             # the grouped GEMM: two launches per step, 2*R*d*F flops each
             launch_ms = per["expert_ffn"]["ms"] / 2
             # the library takes 2-CTA pair tiles when R_max / E >= 1024
-            pair = w.dtype == "bf16" and w.T * w.k >= 1024 * w.E
+            pair = w.dtype == "bf16" and w.T * w.k >= 1024 * w.E and not layer.fused
             roof = {"bound": "tensor", "kernel": "gemm_tc2_kernel" if pair else "gemm_tc_kernel",
                     "achieved": 2.0 * R_mean * w.d * w.F / (launch_ms * 1e-3) / 1e12,
                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
@@ -584,7 +594,7 @@ def main():
         roof["peak_source"] = (
             "derived fp32 FMA peak: 148 x 128 x 2 x sm_max_mhz" if roof["bound"] == "alu" else
             f"{peak_src} ({'bf16_tflops_sustained' if roof['unit'] == 'TFLOP/s' else 'hbm_gbs'})")
-        roof["traffic"] = (gemm_traffic(w.name, roof["kernel"])
+        roof["traffic"] = (gemm_traffic(w.name + ("/fused" if layer.fused else ""), roof["kernel"])
                            if roof["kernel"].startswith("gemm_tc") and args.tokens == 0
                            and args.experts == 0 else None)
         value = w.T * steps * world / (elapsed_ms * 1e-3)
@@ -598,7 +608,7 @@ def main():
                 "n_gpus": world, "steps": steps, "warmup": warmup,
                 "ms_per_step": elapsed_ms / steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-                "config": config_of(w, world),
+                "config": config_of(w, world, layer.fused),
                 "e2e": {"value": w.T * e2e_steps * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": layer.launches_per_forward(gate=not w.logits_direct) * steps,

@@ -182,13 +182,33 @@ MOE_API int moe_expert_ffn(const void* Xp, const void* W1, const void* W2, int d
                    int F, const int32_t* offsets, int R_max, void* H, void* Yp,
                    moe_stream_t stream);
 
+/* Expert computation fused with input encode and the gate weights (ScatterMoE
+ * style; "A Survey on Mixture of Experts", section 5 names the encode/decode
+ * memory traffic as MoE overhead).  bf16 only, tcgen05 tensor cores:
+ *   H[r][f]  = max(0, sum_c x[t(r)][c] * W1[e][f][c]),  t(r) = row_slot[r] / k
+ *              (the A tiles are gathered from x directly: no Xp is written)
+ *   Yp[r][o] = s(r) * sum_f H[r][f] * W2[e][o][f],  s(r) = w[row_slot[r]]
+ *              (w = NULL: s = 1, i.e. moe_expert_ffn's Yp)
+ * for the rows r of each group e.  Output decode is then a plain sum of each
+ * token's rows: moe_combine with w = NULL.  x [T, d]; row_slot [R_max] and
+ * offsets [E+1] from moe_route; w [T, k] from moe_route or NULL; H [R_max, F];
+ * Yp [R_max, d].  Rounding: the scaled fp32 sum is rounded once to bf16.
+ * row_slot entries outside [0, T*k) are flagged (MOE_DEVERR_ROW_INDEX) and
+ * read as zero rows.  fp32 layers: MOE_ERR_UNSUPPORTED.
+ */
+MOE_API int moe_expert_ffn_gather(const void* x, int T, int k, const int32_t* row_slot,
+                                  const float* w, const void* W1, const void* W2, int dtype, int E,
+                                  int d, int F, const int32_t* offsets, int R_max, void* H,
+                                  void* Yp, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- a4 ----
  * Output decode.  "A Survey on Mixture of Experts", section 5: the inverse of
  * input encode restores token order by the gating indices; each token's
  * output is the gate-weighted sum of its experts' outputs:
  *   y[t] = sum_{j < k, slot_row[t][j] >= 0} w[t][j] * Yp[slot_row[t][j]]
  *   accumulated in fp32 with j ascending, rounded once to dtype.  A token
- *   whose slots were all dropped gets zeros.
+ *   whose slots were all dropped gets zeros.  w = NULL: unit weights (the
+ *   rows already carry them, as moe_expert_ffn_gather writes them).
  *   Yp [R_max, d] dtype; slot_row, w [T, k]; y [T, d] dtype.
  */
 MOE_API int moe_combine(const void* Yp, int dtype, int T, int d, int k, const int32_t* slot_row,

@@ -1,5 +1,5 @@
-// ffn.cu -- moe_expert_ffn and moe_gate entry points (argument checks, then
-// the grouped GEMM launches).
+// ffn.cu -- moe_expert_ffn, moe_expert_ffn_gather and moe_gate entry points
+// (argument checks, then the grouped GEMM launches).
 //
 // Expert computation, PopFetcher section 5.1: FC(d -> F), ReLU, FC(F -> d),
 // run group by group over the contiguous per-expert row blocks of input
@@ -36,6 +36,27 @@ extern "C" MOE_API int moe_expert_ffn(const void* Xp, const void* W1, const void
     if (rc != MOE_OK) return rc;
     return launch_gemm_simt_f32(static_cast<const float*>(H), static_cast<const float*>(W2),
                                 static_cast<float*>(Yp), d, F, E, offsets, 0, R_max, false, st);
+}
+
+extern "C" MOE_API int moe_expert_ffn_gather(const void* x, int T, int k, const int32_t* row_slot,
+                                             const float* w, const void* W1, const void* W2,
+                                             int dtype, int E, int d, int F,
+                                             const int32_t* offsets, int R_max, void* H, void* Yp,
+                                             moe_stream_t stream) {
+    if (!dtype_ok(dtype)) return MOE_ERR_UNSUPPORTED;
+    if (dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;  // tensor-core path only
+    if (T < 0 || k < 1 || k > kMaxTopK || E < 1 || E > kMaxExperts || d < 1 || F < 1 || R_max < 0)
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)T * k >= INT32_MAX || (int64_t)E * d >= INT32_MAX || (int64_t)E * F >= INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (R_max > 0 && (!x || !row_slot || !W1 || !W2 || !offsets || !H || !Yp))
+        return MOE_ERR_INVALID_ARG;
+    if ((d * 2) % 16 != 0 || (F * 2) % 16 != 0) return MOE_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(W1) || !aligned16(W2) || !aligned16(H) || !aligned16(Yp))
+        return MOE_ERR_UNSUPPORTED;
+    if (R_max == 0 || T == 0) return MOE_OK;
+    return launch_ffn_gather_bf16(x, T, k, row_slot, w, W1, W2, E, d, F, offsets, R_max, H, Yp,
+                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" MOE_API int moe_gate(const void* x, const void* Wg, int dtype, int T, int d, int E,

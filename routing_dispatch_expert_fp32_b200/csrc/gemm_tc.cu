@@ -19,7 +19,17 @@
 //              row-masked 16-byte stores (rows past the group end belong to
 //              the next group and are never written).
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap the
-// mainloop of tile i+1.  Every mbarrier wait is bounded in time: on expiry the
+// mainloop of tile i+1.
+//
+// Fused variants (ScatterMoE-style, "A Survey on Mixture of Experts",
+// section 5; no dispatched copy of the tokens):
+//   MODE_GATHER   the A tile's 128 rows are gathered straight from the token
+//                 matrix x: grouped row r reads x[row_slot[r] / k], four rows
+//                 per TMA tile::gather4 load, the 32 producer lanes issuing one
+//                 each (rows past the group read out of bounds: zeros);
+//   MODE_ROW_W    the epilogue scales grouped row r by its gate weight
+//                 w[row_slot[r]] before rounding, so output decode becomes a
+//                 plain sum of each token's rows.  Every mbarrier wait is bounded in time: on expiry the
 // kernel flags MOE_DEVERR_TIMEOUT, drains its own TMA loads and MMAs, frees
 // TMEM and returns.
 #include "grouped.cuh"
@@ -51,11 +61,31 @@ struct Cfg {
 };
 
 // -------------------------------------------------------------------- kernel
-template <int BN_MAX, bool RELU, typename TOut>
+enum Mode { MODE_PLAIN = 0, MODE_GATHER = 1, MODE_ROW_W = 2 };
+
+// Row-gather description for the fused modes: grouped row r is slot
+// row_slot[r] = t * k + j of token t; w (MODE_ROW_W) is indexed by the slot.
+struct Gather {
+    const int32_t* row_slot;
+    const float* w;
+    int k, T;
+};
+
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y0, int y1, int y2, int y3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
+        "r"(y2), "r"(y3)
+        : "memory");
+}
+
+template <int BN_MAX, bool RELU, typename TOut, int MODE = MODE_PLAIN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                TOut* __restrict__ C, int N, int K, int E, const int32_t* __restrict__ offsets,
-               int single_M, int R_max, int32_t* err) {
+               int single_M, int R_max, Gather gat, int32_t* err) {
     using G = Cfg<BN_MAX>;
     constexpr int S = G::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -106,7 +136,60 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     const uint32_t tmem_base = *tmem_slot;
     const int nk = (K + BK - 1) / BK;
 
-    if (warp == 0) {
+    if (warp == 0 && MODE == MODE_GATHER) {
+        // -------------------------------------------- TMA producer (gather)
+        // lane l owns tile rows 4l .. 4l+3: their x rows are looked up once
+        // per tile, then every k-block each lane issues one gather4
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)));
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)));
+        }
+        int stage = 0;
+        uint32_t phase = 0;
+        long long issued = 0;
+        bool ok = true;
+        const int n_slots = gat.T * gat.k;
+        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            const TileCoord c = tile_coord(tile, s_prefix, E, offsets, single_M, BM, bn, nt);
+            const int b_row = c.e * N + c.n0;
+            int xr[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = 4 * lane + j;
+                xr[j] = gat.T;  // out of bounds: the TMA fills zeros
+                if (i < c.rows) {
+                    const int slot = __ldg(gat.row_slot + c.row0 + i);
+                    if (slot >= 0 && slot < n_slots) xr[j] = slot / gat.k;
+                    else flag_error(err, MOE_DEVERR_ROW_INDEX);
+                }
+            }
+            for (int kb = 0; kb < nk; ++kb) {
+                int w_ok = 1;
+                if (lane == 0) {
+                    w_ok = mbar_wait(empty + stage, phase ^ 1u, abort_flag, err);
+                    if (w_ok) mbar_arrive_expect_tx(full + stage, stage_tx);
+                }
+                if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+                    ok = false;
+                    break;
+                }
+                tma_gather4(sA + stage * G::A_BYTES + lane * 512, &tmap_a, full + stage, kb * BK,
+                            xr[0], xr[1], xr[2], xr[3]);
+                if (lane == 0)
+                    tma_load_2d(sB + stage * G::B_BYTES, &tmap_b, full + stage, kb * BK, b_row);
+                ++issued;
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            const long long n = issued < S ? issued : S;
+            for (long long i = issued - n; i < issued; ++i)
+                mbar_wait(full + (int)(i % S), (uint32_t)((i / S) & 1), abort_flag, err, false);
+        }
+    } else if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
             const CUtensorMap* mb = &tmap_b;
@@ -191,10 +274,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
             tc_fence_after();
             const bool row_ok = row < c.rows;
             TOut* crow = C + static_cast<size_t>(c.row0 + (row_ok ? row : 0)) * N;
+            float wr = 1.0f;  // MODE_ROW_W: this row's gate weight
+            if (MODE == MODE_ROW_W && row_ok) {
+                const int slot = __ldg(gat.row_slot + c.row0 + row);
+                if (slot >= 0 && slot < gat.T * gat.k) wr = __ldg(gat.w + slot);
+                else flag_error(err, MOE_DEVERR_ROW_INDEX);
+            }
 #pragma unroll 1
             for (int cc = 0; cc < bn; cc += 32) {
                 uint32_t r[32];
                 tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN_MAX + cc), r);
+                if (MODE == MODE_ROW_W) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r[i] = __float_as_uint(__fmul_rn(wr, __uint_as_float(r[i])));
+                }
                 const int col = c.n0 + cc;
                 if (row_ok && col < N) Store32<TOut, RELU>::run(crow + col, r, N - col);
             }
@@ -469,22 +563,27 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
 }  // namespace pair
 
 // -------------------------------------------------------------------- host --
-template <int BN, bool RELU, typename TOut>
+template <int BN, bool RELU, typename TOut, int MODE = MODE_PLAIN>
 static int launch(const void* A, const void* B, TOut* C, int N, int K, int E,
-                  const int32_t* offsets, int single_M, int R_max, cudaStream_t st) {
+                  const int32_t* offsets, int single_M, int R_max, cudaStream_t st,
+                  Gather gat = Gather{nullptr, nullptr, 1, 0}) {
     using G = Cfg<BN>;
     if (R_max <= 0 || N <= 0) return MOE_OK;
     CUtensorMap ta, tb;
-    if (make_tmap(&ta, A, K, R_max, BM) != MOE_OK) return MOE_ERR_CUDA;
+    if (MODE == MODE_GATHER) {  // A = the token matrix x [T, K], one-row boxes
+        if (make_tmap(&ta, A, K, gat.T, 1) != MOE_OK) return MOE_ERR_CUDA;
+    } else if (make_tmap(&ta, A, K, R_max, BM) != MOE_OK) {
+        return MOE_ERR_CUDA;
+    }
     if (make_tmap(&tb, B, K, E * N, BN) != MOE_OK) return MOE_ERR_CUDA;
     const int smem = G::smem_bytes(E);
-    auto kern = gemm_tc_kernel<BN, RELU, TOut>;
-    if (ensure_smem<gemm_tc_kernel<BN, RELU, TOut>>(smem) != MOE_OK) return MOE_ERR_CUDA;
+    auto kern = gemm_tc_kernel<BN, RELU, TOut, MODE>;
+    if (ensure_smem<gemm_tc_kernel<BN, RELU, TOut, MODE>>(smem) != MOE_OK) return MOE_ERR_CUDA;
     const int nt = (N + BN - 1) / BN;
     const long long ub = ((long long)R_max / BM + E) * nt;
     const int grid = (int)(ub < num_sms() ? ub : num_sms());
     return launch_pdl(kern, grid, kThreads, smem, st, ta, tb, C, N, K, E, offsets, single_M, R_max,
-                      device_error_word());
+                      gat, device_error_word());
 }
 
 template <bool RELU>
@@ -528,6 +627,23 @@ int launch_gemm_tc_bf16(const void* A, const void* B, void* C, bool out_f32, int
     }
     if (relu) return launch<256, true, __nv_bfloat16>(A, B, Cb, N, K, E, offsets, single_M, R_max, st);
     return launch<256, false, __nv_bfloat16>(A, B, Cb, N, K, E, offsets, single_M, R_max, st);
+}
+
+int launch_ffn_gather_bf16(const void* x, int T, int k, const int32_t* row_slot, const float* w,
+                           const void* W1, const void* W2, int E, int d, int F,
+                           const int32_t* offsets, int R_max, void* H, void* Yp,
+                           cudaStream_t st) {
+    using namespace tc;
+    const Gather g{row_slot, w, k, T};
+    __nv_bfloat16* Hb = static_cast<__nv_bfloat16*>(H);
+    __nv_bfloat16* Yb = static_cast<__nv_bfloat16*>(Yp);
+    int rc = launch<256, true, __nv_bfloat16, MODE_GATHER>(x, W1, Hb, F, d, E, offsets, 0, R_max,
+                                                           st, g);
+    if (rc != MOE_OK) return rc;
+    if (w != nullptr)
+        return launch<256, false, __nv_bfloat16, MODE_ROW_W>(H, W2, Yb, d, F, E, offsets, 0,
+                                                             R_max, st, g);
+    return launch<256, false, __nv_bfloat16>(H, W2, Yb, d, F, E, offsets, 0, R_max, st);
 }
 
 }  // namespace moe

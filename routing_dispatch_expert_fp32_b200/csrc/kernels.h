@@ -6,6 +6,14 @@
 
 namespace moe {
 
+// Expert FFN with the token rows gathered straight from x (no dispatched
+// copy) and, when w is non-null, the gate weight applied to each output row
+// (gemm_tc.cu, bf16, 1-CTA tiles).
+int launch_ffn_gather_bf16(const void* x, int T, int k, const int32_t* row_slot, const float* w,
+                           const void* W1, const void* W2, int E, int d, int F,
+                           const int32_t* offsets, int R_max, void* H, void* Yp,
+                           cudaStream_t st);
+
 // fp32 grouped GEMM on the CUDA cores (gemm_simt.cu).
 int launch_gemm_simt_f32(const float* A, const float* B, float* C, int N, int K, int E,
                          const int32_t* offsets, int single_M, int R_max, bool relu,

@@ -185,7 +185,7 @@ extern "C" MOE_API int moe_combine(const void* Yp, int dtype, int T, int d, int 
                            const float* w, void* y, int R_max, moe_stream_t stream) {
     const int rc = check_rows(Yp, y, dtype, T, d, k);
     if (rc != MOE_OK) return rc;
-    if (T > 0 && (!slot_row || !w || R_max < 0)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!slot_row || R_max < 0)) return MOE_ERR_INVALID_ARG;  // w NULL: unit weights
     if (T == 0) return MOE_OK;
     const int nvec = (int)((size_t)d * dtype_bytes(dtype) / 16);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -38,6 +38,8 @@ _SIGS = {
     "moe_dispatch": ([_p, _i, _i, _i, _i, _p, _p, _i, _p], _i),
     "moe_expert_ffn": ([_p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _p, _p], _i),
     "moe_combine": ([_p, _i, _i, _i, _i, _p, _p, _p, _i, _p], _i),
+    "moe_expert_ffn_gather": ([_p, _i, _i, _p, _p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _p, _p],
+                              _i),
     "moe_popularity_update": ([_p, _i, _p, _i, _i64, _p, _i, _p, _p], _i),
     "moe_popularity_update_dev": ([_p, _i, _p, _i, _p, _p, _i, _p, _p], _i),
     "moe_route_noalloc": ([_p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i),
@@ -127,6 +129,15 @@ def moe_expert_ffn(Xp, W1, W2, offsets, H, Yp, stream=None):
     _check("moe_expert_ffn", lib.moe_expert_ffn(
         _ptr(Xp), _ptr(W1), _ptr(W2), dtype_code(Xp), E, d, F, _ptr(offsets), Xp.shape[0],
         _ptr(H), _ptr(Yp), _stream(stream)))
+
+
+def moe_expert_ffn_gather(x, k, row_slot, w, W1, W2, offsets, H, Yp, stream=None):
+    """Expert FFN on rows gathered from x by row_slot; w (or None) scales each row."""
+    T, d = x.shape
+    E, F, _ = W1.shape
+    _check("moe_expert_ffn_gather", lib.moe_expert_ffn_gather(
+        _ptr(x), T, k, _ptr(row_slot), _ptr(w), _ptr(W1), _ptr(W2), dtype_code(x), E, d, F,
+        _ptr(offsets), H.shape[0], _ptr(H), _ptr(Yp), _stream(stream)))
 
 
 def moe_combine(Yp, k, slot_row, w, y, stream=None):
@@ -232,10 +243,14 @@ class MoELayer:
     """
 
     def __init__(self, T, d, E, k, F, dtype, capacity=0, W=4, P=8, device="cuda",
-                 identity_experts=False):
+                 identity_experts=False, fused=False):
         self.T, self.d, self.E, self.k, self.F = T, d, E, k, F
         self.dtype, self.capacity, self.W, self.P = dtype, capacity, W, P
         self.identity_experts = identity_experts
+        # fused: the first expert GEMM gathers its rows from x and the second
+        # applies the gate weights (no dispatch pass, combine is a plain sum);
+        # bf16 layers with experts only, forward only
+        self.fused = bool(fused) and not identity_experts and dtype == torch.bfloat16
         dev, i32 = device, torch.int32
         Rmax = max(T * k, 1)
         self.logits = torch.empty(T, E, dtype=torch.float32, device=dev)
@@ -271,6 +286,11 @@ class MoELayer:
                 counts_hook(self.counts)
             moe_popularity_update_dev(self.counts, self.hist, self.step_dev, self.mean, self.P,
                                       self.hot, stream)
+        if self.fused:
+            moe_expert_ffn_gather(x, self.k, self.row_slot, self.w, W1, W2, self.offsets, self.H,
+                                  self.Yp, stream)
+            moe_combine(self.Yp, self.k, self.slot_row, None, self.y, stream)
+            return self.y
         moe_dispatch(x, self.k, self.slot_row, self.Xp, stream)
         if not self.identity_experts:
             moe_expert_ffn(self.Xp, W1, W2, self.offsets, self.H, self.Yp, stream)
@@ -285,6 +305,8 @@ class MoELayer:
         dlogits, dbias and (when ``weight_grads``) dW1, dW2, dWg; dWg and the
         gate's share of dx only when Wg is given (the forward ran the gate).
         """
+        if self.fused:
+            raise RuntimeError("backward needs the unfused forward (Xp and unweighted Yp)")
         T, d, E, k, F = self.T, self.d, self.E, self.k, self.F
         dev = self.y.device
         if not hasattr(self, "dYp"):
@@ -365,7 +387,8 @@ class MoELayer:
 
     def launches_per_forward(self, gate=True, popularity=True) -> int:
         """Kernel launches one forward makes (route is three kernels)."""
-        n = 3 + 1 + 1  # route, dispatch, combine
+        n = 3 + 1  # route, combine
+        n += 0 if self.fused else 1  # dispatch
         n += 1 if gate else 0
         n += 1 if popularity else 0
         n += 0 if self.identity_experts else 2

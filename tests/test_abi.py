@@ -87,7 +87,7 @@ def test_dispatch_combine_reject_bad_arguments(lib):
     assert d(FAKE, 1, 4, 64, 33, FAKE, FAKE, 8, None) == -1         # k > 32
     assert d(FAKE, 1, 0, 64, 2, FAKE, FAKE, 0, None) == 0            # T = 0 is a no-op
     c = lib.moe_combine
-    assert c(FAKE, 1, 4, 64, 2, FAKE, None, FAKE, 8, None) == -1    # w missing
+    assert c(FAKE, 1, 4, 64, 2, None, FAKE, FAKE, 8, None) == -1    # slot_row missing
     assert c(FAKE, 0, 4, 6, 2, FAKE, FAKE, FAKE, 8, None) == -2     # 24-byte fp32 rows
 
 
@@ -97,6 +97,14 @@ def test_ffn_gate_popularity_reject_bad_arguments(lib):
     assert f(FAKE, FAKE, FAKE, 1, 0, 64, 64, FAKE, 8, FAKE, FAKE, None) == -1
     assert f(FAKE, FAKE, FAKE, 1, 4, 64, 64, None, 8, FAKE, FAKE, None) == -1
     assert f(FAKE, FAKE, FAKE, 1, 4, 64, 64, FAKE, 0, FAKE, FAKE, None) == 0    # nothing to do
+    fg = lib.moe_expert_ffn_gather
+    fg.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P, P] + [ctypes.c_int] * 4 + \
+        [P, ctypes.c_int, P, P, P]
+    assert fg(FAKE, 16, 2, FAKE, FAKE, FAKE, FAKE, 0, 4, 64, 64, FAKE, 32, FAKE, FAKE, None) == -2
+    assert fg(FAKE, 16, 0, FAKE, FAKE, FAKE, FAKE, 1, 4, 64, 64, FAKE, 32, FAKE, FAKE, None) == -1
+    assert fg(FAKE, 16, 2, None, FAKE, FAKE, FAKE, 1, 4, 64, 64, FAKE, 32, FAKE, FAKE, None) == -1
+    assert fg(FAKE, 16, 2, FAKE, None, FAKE, FAKE, 1, 4, 60, 64, FAKE, 32, FAKE, FAKE, None) == -2
+    assert fg(FAKE, 0, 2, FAKE, None, FAKE, FAKE, 1, 4, 64, 64, FAKE, 32, FAKE, FAKE, None) == 0
     g = lib.moe_gate
     assert g(FAKE, FAKE, 1, 8, 12, 4, FAKE, None) == -2                          # 24-byte rows
     assert g(FAKE, FAKE, 1, 0, 64, 4, FAKE, None) == 0
