@@ -50,6 +50,12 @@ def parse():
     ap.add_argument("--experts", type=int, default=0,
                     help="override E (smaller profiling cases of the same shapes)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--concurrent", type=int, default=0,
+                    help="independent batches in flight on one GPU (one stream each, one CUDA "
+                         "graph, popularity updates in order); 1 = one batch at a time; "
+                         "0 = by size: 3 when the expert GEMMs of a step are under 0.2 TFLOP "
+                         "(their waves leave SMs idle that another batch's kernels fill), 2 for "
+                         "identity experts, else 1 (measured slower there)")
     ap.add_argument("--path", default="unfused", choices=["unfused", "fused"],
                     help="fused: gather the first GEMM's rows from x and weight the second "
                          "GEMM's rows (no dispatch pass); bf16 expert layers only")
@@ -399,8 +405,42 @@ def main():
         else:
             step(i)
 
+    # Concurrent batches (single rank, graphs): `conc` layer instances with
+    # their own buffers and one shared popularity window; group g runs
+    # batches g*conc .. g*conc+conc-1 (mod nb), one per stream, in one graph.
+    conc = args.concurrent
+    if conc <= 0:
+        if w.identity_experts:
+            conc = 2
+        else:
+            conc = 3 if 4.0 * w.T * w.k * w.d * w.F < 2e11 else 1
+    conc = conc if use_graph else 1
+    layers = [layer]
+    groups, group_batches = [], []
+    if conc > 1:
+        for _ in range(conc - 1):
+            extra = moe.MoELayer(w.T, w.d, w.E, w.k, w.F, tdt, capacity=w.capacity, W=w.W,
+                                 P=w.P, identity_experts=w.identity_experts,
+                                 fused=args.path == "fused")
+            extra.share_popularity(layer)
+            layers.append(extra)
+        for g in range(max(1, nb // conc)):
+            idx = [(g * conc + i) % nb for i in range(conc)]
+            calls = [dict(x=batches[j]["x"], Wg=weights.get("Wg"), W1=weights.get("W1"),
+                          W2=weights.get("W2"), bias=batches[j]["bias"],
+                          logits=batches[j].get("logits")) for j in idx]
+            groups.append(moe.capture_concurrent(layers, calls))
+            group_batches.append(idx)
+        steps = (steps + conc - 1) // conc * conc  # whole groups
+
+    def run_group(g):
+        groups[g % len(groups)].replay()
+
     for i in range(warmup):
-        run_step(i)
+        if conc > 1:
+            run_group(i)
+        else:
+            run_step(i)
     torch.cuda.synchronize()
 
     def barrier():
@@ -416,8 +456,12 @@ def main():
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for i in range(steps):
-        run_step(i)
+    if conc > 1:
+        for g in range(steps // conc):
+            run_group(g)
+    else:
+        for i in range(steps):
+            run_step(i)
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
@@ -427,6 +471,20 @@ def main():
         t = torch.tensor([elapsed_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         elapsed_ms = float(t.item())
+    # one batch at a time (the single-stream graphs), for comparison
+    seq = None
+    if conc > 1:
+        seq_steps = min(steps, 1000)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        s0.record(stream)
+        for i in range(seq_steps):
+            run_step(i)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        seq_ms = s0.elapsed_time(s1)
+        seq = {"value": w.T * seq_steps / (seq_ms * 1e-3), "ms_per_step": seq_ms / seq_steps,
+               "steps": seq_steps, "note": "the same graphs replayed one batch at a time"}
 
     # ---- timed region 2: the same calls issued one by one with an event after
     # each stage: per-stage device times and the kernels' roofline numbers ----
@@ -458,30 +516,91 @@ def main():
 
     def e2e_step(i):
         b = batches[i % nb]
-        if use_graph:  # the graph reads the batch's own device buffers
-            b["x"].copy_(host_x[i % nb], non_blocking=True)
-            if dlog is not None:
-                b["logits"].copy_(host_logits[i % nb], non_blocking=True)
-            graphs[i % nb].replay()
-        else:
-            dx.copy_(host_x[i % nb], non_blocking=True)
-            if dlog is not None:
-                dlog.copy_(host_logits[i % nb], non_blocking=True)
-            layer.forward(dx, weights.get("Wg"), weights.get("W1"), weights.get("W2"), b["bias"],
-                          logits=dlog, counts_hook=hook)
+        dx.copy_(host_x[i % nb], non_blocking=True)
+        if dlog is not None:
+            dlog.copy_(host_logits[i % nb], non_blocking=True)
+        layer.forward(dx, weights.get("Wg"), weights.get("W1"), weights.get("W2"), b["bias"],
+                      logits=dlog, counts_hook=hook)
         host_y.copy_(layer.y, non_blocking=True)
 
-    for i in range(3):
-        e2e_step(i)
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
+    e2e_pipelined = use_graph
+    if e2e_pipelined:
+        # Two units, each a graph over `conc` batches with its own layer
+        # instances and device input buffers; copies run on their own streams
+        # so unit u's inputs arrive and unit u-1's outputs leave while the
+        # other unit computes (every step still copies its x in and its y out).
+        def make_unit(unit_layers, first):
+            idx = [(first + i) % nb for i in range(len(unit_layers))]
+            xs = [batches[j]["x"].clone() for j in idx]
+            lg = [None if batches[j].get("logits") is None else batches[j]["logits"].clone()
+                  for j in idx]
+            calls = [dict(x=xs[i], Wg=weights.get("Wg"), W1=weights.get("W1"),
+                          W2=weights.get("W2"), bias=batches[j]["bias"], logits=lg[i])
+                     for i, j in enumerate(idx)]
+            if len(unit_layers) > 1:
+                g = moe.capture_concurrent(unit_layers, calls)
+            else:
+                g = unit_layers[0].capture(**calls[0])
+            hy = [torch.empty(w.T, w.d, dtype=tdt).pin_memory() for _ in unit_layers]
+            return dict(graph=g, idx=idx, xs=xs, lg=lg, layers=unit_layers, hy=hy,
+                        comp=None, out=None)
+
+        second = []
+        for _ in range(conc):
+            extra = moe.MoELayer(w.T, w.d, w.E, w.k, w.F, tdt, capacity=w.capacity, W=w.W,
+                                 P=w.P, identity_experts=w.identity_experts,
+                                 fused=args.path == "fused")
+            extra.share_popularity(layer)
+            second.append(extra)
+        units = [make_unit(layers, 0), make_unit(second, conc % nb)]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+        def e2e_unit(it):
+            u = units[it % 2]
+            if u["comp"] is not None:
+                s_in.wait_event(u["comp"])  # the unit's previous replay has read its inputs
+            with torch.cuda.stream(s_in):
+                for i, j in enumerate(u["idx"]):
+                    u["xs"][i].copy_(host_x[j], non_blocking=True)
+                    if u["lg"][i] is not None:
+                        u["lg"][i].copy_(host_logits[j], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+            stream.wait_event(ev_in)
+            if u["out"] is not None:
+                stream.wait_event(u["out"])  # its previous outputs have left
+            u["graph"].replay()
+            u["comp"] = torch.cuda.Event()
+            u["comp"].record(stream)
+            s_out.wait_event(u["comp"])
+            with torch.cuda.stream(s_out):
+                for L, hy in zip(u["layers"], u["hy"]):
+                    hy.copy_(L.y, non_blocking=True)
+                u["out"] = torch.cuda.Event()
+                u["out"].record(s_out)
+
+        e2e_steps = (e2e_steps + conc - 1) // conc * conc
+        for it in range(4):
+            e2e_unit(it)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s_in)
+        for it in range(e2e_steps // conc):
+            e2e_unit(it)
+        e1.record(s_out)
+        torch.cuda.synchronize()
+    else:
+        for i in range(3):
+            e2e_step(i)
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
     e2e_ms = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([e2e_ms], device="cuda")
@@ -608,13 +727,20 @@ def main():
                 "n_gpus": world, "steps": steps, "warmup": warmup,
                 "ms_per_step": elapsed_ms / steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-                "config": config_of(w, world, layer.fused),
+                "config": dict(config_of(w, world, layer.fused), batches_in_flight=conc),
                 "e2e": {"value": w.T * e2e_steps * world / (e2e_ms * 1e-3), "unit": "tokens/s",
-                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                        "note": ("pinned host x in and y out every step, on copy streams that "
+                                 "overlap the other of two alternating graph units"
+                                 if e2e_pipelined else
+                                 "pinned host x in and y out every step, in stream order")},
                 "gpu_launches": layer.launches_per_forward(gate=not w.logits_direct) * steps,
                 "roofline": roof, "stages": per, "clocks": clocks, "cpu_baseline": cpu,
-                "timing": {"value": "CUDA-graph replay of the whole step" if use_graph
+                "timing": {"value": (f"CUDA-graph replay, {conc} independent batches in flight "
+                                     "(one stream each, popularity updates in order)")
+                           if conc > 1 else "CUDA-graph replay of the whole step" if use_graph
                            else "kernels issued one by one (programmatic dependent launch)",
+                           "one_batch_at_a_time": seq,
                            "stages_and_roofline": f"{stage_steps} steps issued stage by stage, "
                                                   "events between stages"},
                 "extras": extras, "device_error_bits": dev_err}

@@ -273,8 +273,15 @@ class MoELayer:
         self.hot = torch.empty(max(P, 1), dtype=i32, device=dev)
         self.step_dev = torch.zeros(1, dtype=torch.int64, device=dev)
 
+    def share_popularity(self, other: "MoELayer"):
+        """Use other's popularity window (ring, step counter, mean, hot): two
+        instances that run batches of the same layer concurrently keep one
+        window, provided their updates are ordered (see capture_concurrent)."""
+        self.hist, self.mean, self.hot, self.step_dev = (other.hist, other.mean, other.hot,
+                                                         other.step_dev)
+
     def forward(self, x, Wg=None, W1=None, W2=None, bias=None, logits=None, stream=None,
-                popularity=True, counts_hook=None):
+                popularity=True, counts_hook=None, popularity_done=None):
         if logits is None:
             moe_gate(x, Wg, self.logits, stream)
             logits = self.logits
@@ -286,6 +293,8 @@ class MoELayer:
                 counts_hook(self.counts)
             moe_popularity_update_dev(self.counts, self.hist, self.step_dev, self.mean, self.P,
                                       self.hot, stream)
+            if popularity_done is not None:
+                popularity_done()
         if self.fused:
             moe_expert_ffn_gather(x, self.k, self.row_slot, self.w, W1, W2, self.offsets, self.H,
                                   self.Yp, stream)
@@ -393,3 +402,40 @@ class MoELayer:
         n += 1 if popularity else 0
         n += 0 if self.identity_experts else 2
         return n
+
+
+def capture_concurrent(layers, calls):
+    """One CUDA graph that runs ``layers[i].forward(**calls[i])`` for every i,
+    each on a stream of its own, so independent batches overlap on the GPU
+    (small kernels of one batch fill SMs the other batch's GEMM waves leave
+    idle).  Layers that share a popularity window (``share_popularity``) get
+    their updates ordered in list order.  Capturing runs every forward once
+    (torch's warm-up), which advances the window."""
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side.wait_stream(main)
+    with torch.cuda.stream(side):
+        for layer, call in zip(layers, calls):
+            layer.forward(**call)
+    main.wait_stream(side)
+    streams = [torch.cuda.Stream() for _ in layers]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cap = torch.cuda.current_stream()
+        prev = None
+        for layer, call, st in zip(layers, calls, streams):
+            st.wait_stream(cap)
+            done = torch.cuda.Event()
+            with torch.cuda.stream(st):
+                def before(counts, wait_for=prev):
+                    if wait_for is not None:
+                        torch.cuda.current_stream().wait_event(wait_for)
+
+                def after(ev=done):
+                    ev.record(torch.cuda.current_stream())
+
+                layer.forward(**call, counts_hook=before, popularity_done=after)
+            prev = done
+        for st in streams:
+            cap.wait_stream(st)
+    return graph
