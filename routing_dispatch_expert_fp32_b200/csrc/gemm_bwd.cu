@@ -266,24 +266,31 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 uint8_t* a_st = sA + stage * A_BYTES;
                 uint8_t* b_st = sB + stage * B_BYTES;
                 const int valid = kr - kb * BK;
+                int nsub = BK / 16;  // MMA steps of 16 K-rows this k-block issues
                 if (KVAR && valid < BK) {
-                    // A K-row (or B K-row) is 128 bytes of one box whatever
-                    // the swizzle inside it: zero rows [valid, BK) of A's boxes,
-                    // and of B's too where the block runs past the last
-                    // group (rows no one wrote); inside the buffer B holds the
-                    // next group's finite rows, which the zero A rows cancel
-                    const int per_box = (BK - valid) * 8;  // 16-byte chunks
-                    const bool past_end = k0 + (kb + 1) * BK > s_prefix[E];
-                    const int nbox = BM / MN_BOX + (past_end ? BN / MN_BOX : 0);
-                    const uint4 z = make_uint4(0, 0, 0, 0);
-                    for (int i = lane; i < nbox * per_box; i += 32) {
-                        const int box = i / per_box, q = i - box * per_box;
-                        uint8_t* base = box < BM / MN_BOX
-                                            ? a_st + box * MN_BOX_BYTES
-                                            : b_st + (box - BM / MN_BOX) * MN_BOX_BYTES;
-                        reinterpret_cast<uint4*>(base + valid * 128)[q] = z;
+                    // the group ends inside this block: steps past its end are
+                    // skipped; in the step it ends in, K-rows [valid, 16*nsub)
+                    // are zeroed in A (each K-row is 128 bytes of one box,
+                    // whatever the swizzle inside it), and in B too where the
+                    // rows lie past the last group (rows no one wrote); other B
+                    // rows there belong to the next group, finite, and meet
+                    // zeros in A
+                    nsub = (valid + 15) / 16;
+                    const int zr = nsub * 16 - valid;  // rows to zero
+                    if (zr > 0) {
+                        const bool past_end = k0 + kb * BK + nsub * 16 > s_prefix[E];
+                        const int per_box = zr * 8;  // 16-byte chunks
+                        const int nbox = BM / MN_BOX + (past_end ? BN / MN_BOX : 0);
+                        const uint4 z = make_uint4(0, 0, 0, 0);
+                        for (int i = lane; i < nbox * per_box; i += 32) {
+                            const int box = i / per_box, q = i - box * per_box;
+                            uint8_t* base = box < BM / MN_BOX
+                                                ? a_st + box * MN_BOX_BYTES
+                                                : b_st + (box - BM / MN_BOX) * MN_BOX_BYTES;
+                            reinterpret_cast<uint4*>(base + valid * 128)[q] = z;
+                        }
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                 }
                 if (lane == 0) {
@@ -291,6 +298,7 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const uint32_t b0 = smem_u32(b_st);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
+                        if (kk >= nsub) break;
                         const uint64_t ad =
                             A_MN ? sw128_mn_desc(a0 + kk * 2048) : sw128_desc(a0 + kk * 32);
                         mma_bf16(d_tmem, ad, sw128_mn_desc(b0 + kk * 2048), idesc,
@@ -317,7 +325,6 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int row = quad * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
         uint8_t* stage_c = sC + quad * (kEpiBufs * 4096);  // this warp's staging tiles
-        int nstore = 0;
         int it = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
             int e, m0, rows, n0, k0, nk, kr;
@@ -353,37 +360,47 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
             }
             if (!mbar_wait(tfull + acc, (it >> 1) & 1, abort_flag, err)) break;
             tc_fence_after();
+            if (EPI == EPI_F32) {
+                // fp32 weight gradient: kEpiBufs 32 x 32 blocks of the warp's
+                // rows at a time are staged in shared memory (128-byte swizzle)
+                // behind one proxy fence, then written by one tensor store each;
+                // rows past M_fix and columns past N are clipped by the map
+                const bool rows_in = m0 + quad * 32 < M_fix;
 #pragma unroll 1
-            for (int cc = 0; cc < BN; cc += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + cc), r);
-                const int col = n0 + cc;
-                if (EPI == EPI_F32) {
-                    // fp32 weight gradient: stage the warp's 32 x 32 block in
-                    // shared memory (128-byte swizzle) and store it with one
-                    // tensor store; rows past M_fix and columns past N are
-                    // clipped by the tensor map
-                    if (col >= N || m0 + quad * 32 >= M_fix) continue;  // nothing to store
-                    if (nk == 0) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = 0u;  // group without rows
-                    }
-                    uint8_t* buf = stage_c + (nstore % kEpiBufs) * 4096;
-                    // the store that last used this buffer has read it
-                    if (lane == 0) bulk_wait_read_allow<kEpiBufs - 1>();
+                for (int cb = 0; cb < BN; cb += 32 * kEpiBufs) {
+                    if (lane == 0) bulk_wait_read_allow<0>();  // the last batch has been read
                     __syncwarp();
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        *reinterpret_cast<uint4*>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
-                            make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+                    for (int u = 0; u < kEpiBufs; ++u) {
+                        uint32_t r[32];
+                        tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + cb + 32 * u),
+                                  r);
+                        if (nk == 0) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) r[i] = 0u;  // group without rows
+                        }
+                        uint8_t* buf = stage_c + u * 4096;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            *reinterpret_cast<uint4*>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                                make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+                    }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
-                    if (lane == 0) {
-                        tma_store_3d(&tmap_c, buf, col, m0 + quad * 32, e);
+                    if (lane == 0 && rows_in) {
+                        for (int u = 0; u < kEpiBufs; ++u) {
+                            const int col = n0 + cb + 32 * u;
+                            if (col < N) tma_store_3d(&tmap_c, stage_c + u * 4096, col, m0 + quad * 32, e);
+                        }
                         bulk_commit();
                     }
-                    ++nstore;
-                } else {
+                }
+            } else {
+#pragma unroll 1
+                for (int cc = 0; cc < BN; cc += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + cc), r);
+                    const int col = n0 + cc;
                     const uint32_t mw = hm[0];
 #pragma unroll
                     for (int w = 0; w + 1 < BN / 32; ++w) hm[w] = hm[w + 1];
