@@ -173,3 +173,42 @@ def test_graph_replay_matches_eager_and_advances_the_window(moe):
         assert np.array_equal(host(graphed.hot)[: w.P], hot_ref), s
     assert int(graphed.step_dev.item()) == len(steps)
     assert moe.moe_device_error() == 0
+
+
+def test_concurrent_batches_match_sequential_and_keep_one_window(moe):
+    """capture_concurrent: three batches of one layer on three streams in one
+    graph give each batch the same output as running it alone, and their
+    popularity updates enter the shared window in list order."""
+    w = wl.tiny("conc", T=600, d=256, E=12, k=2, F=384, zipf_s=1.1, W=8, P=4)
+    weights = {k: dev(v) for k, v in wl.make_weights(w).items()}
+    steps = [wl.make_step(w, s) for s in range(3)]
+    xs = [dev(s["x"]) for s in steps]
+    bias = dev(steps[0]["bias"])
+    layers = [make_layer(moe, w) for _ in range(3)]
+    for L in layers[1:]:
+        L.share_popularity(layers[0])
+    calls = [dict(x=x, Wg=weights["Wg"], W1=weights["W1"], W2=weights["W2"], bias=bias)
+             for x in xs]
+    g = moe.capture_concurrent(layers, calls)
+    layers[0].hist.zero_()
+    layers[0].step_dev.zero_()  # the capture's warm-up advanced the window
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    alone = make_layer(moe, w)
+    hist_ref = np.zeros((w.W, w.E), np.int32)
+    s = 0
+    for rep in range(2):
+        for i, x in enumerate(xs):
+            y = alone.forward(x, weights["Wg"], weights["W1"], weights["W2"], bias)
+            torch.cuda.synchronize()
+            if rep == 1:
+                assert torch.equal(layers[i].y, y), i
+            r = oracle.route(host(alone.logits), host(bias), w.k, w.capacity)
+            mean_ref, hot_ref = oracle.popularity_update(r["counts"], hist_ref, s, w.P)
+            s += 1
+    assert int(layers[0].step_dev.item()) == 6
+    assert np.array_equal(host(layers[0].hist), hist_ref)
+    assert np.array_equal(host(layers[0].mean), mean_ref)
+    assert np.array_equal(host(layers[0].hot)[: w.P], hot_ref)
+    assert moe.moe_device_error() == 0
