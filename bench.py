@@ -727,7 +727,7 @@ def main():
                 "n_gpus": world, "steps": steps, "warmup": warmup,
                 "ms_per_step": elapsed_ms / steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-                "config": dict(config_of(w, world, layer.fused), batches_in_flight=conc),
+                "config": config_of(w, world, layer.fused),
                 "e2e": {"value": w.T * e2e_steps * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "note": ("pinned host x in and y out every step, on copy streams that "
@@ -740,6 +740,7 @@ def main():
                                      "(one stream each, popularity updates in order)")
                            if conc > 1 else "CUDA-graph replay of the whole step" if use_graph
                            else "kernels issued one by one (programmatic dependent launch)",
+                           "batches_in_flight": conc,
                            "one_batch_at_a_time": seq,
                            "stages_and_roofline": f"{stage_steps} steps issued stage by stage, "
                                                   "events between stages"},
