@@ -251,13 +251,20 @@ extern "C" MOE_API int moe_expert_ffn_backward(const void* Xp, const void* H, co
     if (!dtype_ok(dtype)) return MOE_ERR_UNSUPPORTED;
     if (E < 1 || E > kMaxExperts || d < 1 || F < 1 || R_max < 0) return MOE_ERR_INVALID_ARG;
     if ((int64_t)E * d >= INT32_MAX || (int64_t)E * F >= INT32_MAX) return MOE_ERR_INVALID_ARG;
-    if (!Xp || !H || !dYp || !W1 || !W2 || !offsets || !dH || !dXp) return MOE_ERR_INVALID_ARG;
+    if (R_max > 0 && (!Xp || !H || !dYp || !W1 || !W2 || !offsets || !dH || !dXp))
+        return MOE_ERR_INVALID_ARG;
     const size_t es = dtype_bytes(dtype);
     if ((d * es) % 16 != 0 || (F * es) % 16 != 0) return MOE_ERR_UNSUPPORTED;
     const void* ptrs[] = {Xp, H, dYp, W1, W2, dH, dXp, dW1, dW2};
     for (const void* p : ptrs)
         if (!aligned16(p)) return MOE_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (R_max == 0) {  // no rows: zero weight gradients, nothing else to do
+        for (float* g : {dW1, dW2})
+            if (g && cudaMemsetAsync(g, 0, sizeof(float) * (size_t)E * d * F, st) != cudaSuccess)
+                return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
     if (dtype == MOE_DTYPE_BF16)
         return launch_ffn_backward_bf16(Xp, H, dYp, W1, W2, E, d, F, offsets, R_max, dH, dXp, dW1,
                                         dW2, st);

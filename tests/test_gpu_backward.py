@@ -314,3 +314,43 @@ def test_ffn_backward_full_size_sampled(moe, name):
     # experts without rows: zero weight gradients
     for e in np.nonzero(np.diff(offsets) == 0)[0]:
         assert not dW1[e].any() and not dW2[e].any()
+
+
+# ------------------------------------------------------------ edge cases ---
+def test_backward_edge_cases(moe):
+    E, d, F, k = 3, 64, 128, 2
+    W1 = dev(rand((E, F, d), 0.1, "bf16", 61))
+    W2 = dev(rand((E, d, F), 0.1, "bf16", 62))
+    z = lambda *s: torch.zeros(*s, dtype=torch.bfloat16, device="cuda")
+    # no rows at all: zero weight gradients
+    dW1 = torch.full((E, F, d), 3.0, device="cuda")
+    dW2 = torch.full((E, d, F), 3.0, device="cuda")
+    offsets = dev(np.zeros(E + 1, np.int32))
+    moe.moe_expert_ffn_backward(z(0, d), z(0, F), z(0, d), W1, W2, offsets, z(0, F), z(0, d),
+                                dW1, dW2)
+    torch.cuda.synchronize()
+    assert not dW1.any() and not dW2.any()
+    # no tokens: route backward gives dbias = 0, gate backward dWg = 0
+    ws = torch.empty(max(moe.moe_route_workspace_size(0, E, k), 1), dtype=torch.uint8,
+                     device="cuda")
+    db = torch.full((E,), 2.0, device="cuda")
+    e_ids = torch.zeros(0, k, dtype=torch.int32, device="cuda")
+    e_f = torch.zeros(0, k, device="cuda")
+    moe.moe_route_backward(e_ids, e_f, e_f, E, torch.zeros(0, E, device="cuda"), db, ws)
+    dWg = torch.full((E, d), 2.0, device="cuda")
+    moe.moe_gate_backward(z(0, d), z(E, d), torch.zeros(0, E, device="cuda"), z(0, d), dWg)
+    torch.cuda.synchronize()
+    assert not db.any() and not dWg.any()
+    # one token, k = E: every expert chosen once, weights sum to one
+    T1 = 1
+    r = oracle.route(np.array([[0.3, -1.0, 2.0]], np.float32), None, E, 0)
+    dw = np.array([[0.5, -2.0, 1.0]], np.float32)
+    dl_r, db_r = oracle.route_backward(r["ids"], r["w"], dw, E)
+    dl = torch.empty(T1, E, device="cuda")
+    db = torch.empty(E, device="cuda")
+    ws = torch.empty(moe.moe_route_workspace_size(T1, E, E), dtype=torch.uint8, device="cuda")
+    moe.moe_route_backward(dev(r["ids"]), dev(r["w"]), dev(dw), E, dl, db, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(dl).view(np.uint32), dl_r.view(np.uint32))
+    assert abs(float(host(dl).astype(np.float64).sum())) < 1e-6  # softmax gradient sums to zero
+    assert moe.moe_device_error() == 0
