@@ -113,3 +113,37 @@ def test_ffn_gate_popularity_reject_bad_arguments(lib):
     assert pu(FAKE, 8, FAKE, 4, 0, FAKE, 9, FAKE, None) == -1                   # P > E
     assert pu(FAKE, 8, FAKE, 0, 0, FAKE, 2, FAKE, None) == -1                   # W = 0
     assert pu(FAKE, 8, FAKE, 4, -1, FAKE, 2, FAKE, None) == -1                  # step < 0
+
+
+def test_backward_entry_points_reject_bad_arguments(lib):
+    i, z = ctypes.c_int, ctypes.c_size_t
+    cb = lib.moe_combine_backward
+    cb.argtypes = [P, P, i, i, i, i, P, P, P, P, i, P]
+    assert cb(FAKE, FAKE, 1, 4, 64, 33, FAKE, FAKE, FAKE, FAKE, 8, None) == -1   # k > 32
+    assert cb(FAKE, FAKE, 0, 4, 6, 2, FAKE, FAKE, FAKE, FAKE, 8, None) == -2     # 24-byte rows
+    assert cb(None, None, 1, 0, 64, 2, None, None, None, None, 0, None) == 0     # T = 0
+    fb = lib.moe_expert_ffn_backward
+    fb.argtypes = [P] * 5 + [i] * 4 + [P, i, P, P, P, P, P]
+    assert fb(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 0, 64, 64, FAKE, 8, FAKE, FAKE, None, None,
+              None) == -1                                                         # E = 0
+    assert fb(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 60, 64, FAKE, 8, FAKE, FAKE, None, None,
+              None) == -2                                                         # d % 8
+    assert fb(None, None, None, FAKE, FAKE, 1, 2, 64, 64, FAKE, 0, None, None, None, None,
+              None) == 0                                                          # no rows
+    db = lib.moe_dispatch_backward
+    db.argtypes = [P, i, i, i, i, P, P, i, P]
+    assert db(FAKE, 1, 4, 64, 40, FAKE, FAKE, 8, None) == -1                     # k > 32
+    rb = lib.moe_route_backward
+    rb.argtypes = [P, P, P, i, i, i, P, P, P, z, P]
+    assert rb(FAKE, FAKE, FAKE, 4, 2, 3, FAKE, None, None, 0, None) == -1        # k > E
+    assert rb(FAKE, FAKE, FAKE, 4, 8, 2, FAKE, FAKE, None, 0, None) == -3        # dbias, no ws
+    assert rb(None, None, None, 0, 8, 2, None, None, None, 0, None) == 0         # T = 0
+    gb = lib.moe_gate_backward
+    gb.argtypes = [P, P, i, i, i, i, P, P, P, P, z, P]
+    assert gb(FAKE, FAKE, 1, 4, 64, 2000, FAKE, FAKE, FAKE, None, 0, None) == -1  # E > 1024
+    assert gb(FAKE, FAKE, 1, 4, 64, 16, FAKE, FAKE, FAKE, None, 0, None) == -3    # dWg, no ws
+    assert gb(None, FAKE, 1, 0, 64, 16, None, None, None, None, 0, None) == 0     # T = 0
+    ws = lib.moe_gate_backward_workspace_size
+    ws.argtypes, ws.restype = [i, i, i, i], z
+    assert ws(4096, 1024, 16, 1) >= 3 * 4096 * 16 * 2  # the three bf16 planes
+    assert ws(0, 1024, 16, 1) == 0
