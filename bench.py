@@ -699,9 +699,17 @@ def main():
         else:
             # the grouped GEMM: two launches per step, 2*R*d*F flops each
             launch_ms = per["expert_ffn"]["ms"] / 2
-            # the library takes 2-CTA pair tiles when R_max / E >= 1024
-            pair = w.dtype == "bf16" and w.T * w.k >= 1024 * w.E and not layer.fused
-            roof = {"bound": "tensor", "kernel": "gemm_tc2_kernel" if pair else "gemm_tc_kernel",
+            # the library takes 2-CTA pair tiles when R_max / E >= 1024 or when
+            # 128-row tiles would fill fewer than three waves of SMs
+            nsm = torch.cuda.get_device_properties(local).multi_processor_count
+
+            def pair_for(N):
+                tiles = (w.T * w.k // 128 + w.E) * ((N + 255) // 256)
+                return (w.dtype == "bf16" and not layer.fused
+                        and (w.T * w.k >= 1024 * w.E or tiles < 3 * nsm))
+            kinds = ["gemm_tc2_kernel" if pair_for(N) else "gemm_tc_kernel" for N in (w.F, w.d)]
+            roof = {"bound": "tensor", "kernel": kinds[0] if kinds[0] == kinds[1]
+                    else "+".join(kinds),
                     "achieved": 2.0 * R_mean * w.d * w.F / (launch_ms * 1e-3) / 1e12,
                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
             if w.dtype == "f32":

@@ -620,8 +620,14 @@ int launch_gemm_tc_bf16(const void* A, const void* B, void* C, bool out_f32, int
     }
     __nv_bfloat16* Cb = static_cast<__nv_bfloat16*>(C);
     // Dense groups (many rows per expert on average) take the 2-CTA 256-row
-    // tiles; sparse ones keep 128-row tiles, which waste fewer padded rows.
-    if (offsets != nullptr && (long long)R_max >= (long long)kPairMinRowsPerGroup * E) {
+    // tiles; sparse ones keep 128-row tiles, which waste fewer padded rows --
+    // unless the 128-row tiles would fill fewer than three waves of SMs, where
+    // halving each SM's weight traffic outweighs the padding (measured on one
+    // B200: the skewed_drops second GEMM, 1.2 waves, 63.2 -> 58.7 us; its first
+    // GEMM, 8.6 waves, and both multistep_window GEMMs are slower with pairs).
+    const long long tiles_1cta = ((long long)R_max / BM + E) * ((N + 255) / 256);
+    if (offsets != nullptr && ((long long)R_max >= (long long)kPairMinRowsPerGroup * E ||
+                               tiles_1cta < 3LL * num_sms())) {
         if (relu) return launch_pair<true>(A, B, Cb, N, K, E, offsets, R_max, st);
         return launch_pair<false>(A, B, Cb, N, K, E, offsets, R_max, st);
     }
