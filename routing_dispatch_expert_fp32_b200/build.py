@@ -58,7 +58,8 @@ def build(force: bool = False, verbose: bool = False, extra=(), out: str = LIB) 
     extra = list(extra)
     if not force and not extra and out == LIB and up_to_date():
         return LIB
-    build_dir = BUILD if not extra else BUILD + "_" + str(abs(hash(tuple(extra))))
+    build_dir = BUILD if not extra else os.path.join(BUILD, "variant_" + "_".join(
+        "".join(c if c.isalnum() else "_" for c in f) for f in extra))
     os.makedirs(build_dir, exist_ok=True)
     with concurrent.futures.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose, extra, build_dir), _sources()))
