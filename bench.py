@@ -229,8 +229,6 @@ def reference_arm(args, w):
     n = 0
     rate = 0.0
     per = args.cpu_seconds / max(1, steps)
-    for _ in range(args.warmup if args.warmup < 3 else 1):
-        pass
     for _ in range(steps):
         rate, n, dt = cpu_oracle_run(w, per)
         times.append(dt)
@@ -239,7 +237,7 @@ def reference_arm(args, w):
             "unit": "tokens/s", "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
-            "data": "synthetic", "config": config_of(w, 1),
+            "data": "synthetic", "config": config_of(w, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": f"first {n} tokens of the batch per step, whole layer"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
