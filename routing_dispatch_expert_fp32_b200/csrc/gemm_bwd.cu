@@ -18,10 +18,15 @@
 // Same pipeline as the forward kernel (gemm_tc.cu): persistent CTAs, TMA
 // producer warp, one MMA-issuing thread, four epilogue warps draining two TMEM
 // accumulators, every wait bounded in time.  For the weight gradients a
-// group's last K block can run past the group's rows; the MMA thread zeroes
-// those K-rows of the A tile in shared memory before issuing (so the products
-// with whatever B holds there vanish).  A group with no rows gets zero weight
-// gradients.
+// group's last K block can run past the group's rows: its 16-row MMA steps
+// past the end are not issued, and in the step where the group ends the MMA
+// warp zeroes the remaining K-rows of A (and of B where they lie past the last
+// group, rows nobody wrote) in shared memory, so that nothing outside the
+// group enters the sum.  A group with no rows gets zero weight gradients.
+// The fp32 weight-gradient tiles leave through shared memory and tensor
+// stores; the bf16 outputs (dH, dXp) are stored row by row, masked to the
+// group.  The same kernel, with a K loop over three planes of A, computes the
+// bf16 gate backward from dlogits split exactly into three bf16 planes.
 #include <cstring>
 
 #include "grouped.cuh"
