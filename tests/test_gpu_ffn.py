@@ -40,6 +40,8 @@ def run_ffn(moe, Xp, W1, W2, offsets, Rmax):
     ([0, 0, 0], 64, 64, "bf16"),
     ([40, 90, 1], 64, 128, "f32"),
     ([0, 65, 200], 72, 100, "f32"),
+    # enough 128-row tiles (>= 3 waves) that the first GEMM stays on 1-CTA tiles
+    ([1000, 1, 0, 1999, 1000], 64, 4096, "bf16"),
 ])
 def test_ffn_small_shapes_elementwise(moe, sizes, d, F, dtype):
     E = len(sizes)
