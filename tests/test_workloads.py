@@ -49,3 +49,20 @@ def test_bf16_conversion_round_trip():
     v = np.array([1.0, -2.5, 3.140625, 1e-30], np.float32)
     assert np.array_equal(wl.bf16_bits_to_f32(wl.to_bf16_bits(v))[:3], v[:3])
     assert wl.to_bf16_bits(np.array([1 + 2 ** -8], np.float32))[0] == 0x3F80
+
+
+def test_backward_generators_are_seeded_and_shaped():
+    w = wl.WORKLOADS["skewed_drops"].with_(T=64, F=32, d=16)
+    a, b = wl.make_grad(w, 1), wl.make_grad(w, 1)
+    assert a.dtype == np.uint16 and a.shape == (64, 16) and np.array_equal(a, b)
+    assert not np.array_equal(a, wl.make_grad(w, 2))
+    inp = wl.ffn_backward_inputs(w, 100)
+    assert inp["Xp"].shape == (100, 16) and inp["dYp"].shape == (100, 16)
+    assert inp["H"].shape == (100, 32)
+    h = wl.bf16_bits_to_f32(inp["H"])
+    assert (h >= 0).all() and 0.3 < (h == 0).mean() < 0.7  # about half zeros, as after a ReLU
+    again = wl.ffn_backward_inputs(w, 100)
+    assert all(np.array_equal(inp[k], again[k]) for k in inp)
+    lg = wl.router_logits(w)
+    assert lg.dtype == np.float32 and lg.shape == (64, w.E)
+    assert np.array_equal(lg, wl.router_logits(w))
