@@ -335,7 +335,9 @@ def main():
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     to_dev = lambda a: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)  # noqa: E731
                         if a.dtype == np.uint16 else torch.from_numpy(a)).cuda()
-    weights = {k: to_dev(v) for k, v in wl.make_weights(w, rank).items()}
+    # one layer replicated on every rank (data parallel): the same weights everywhere,
+    # a differently seeded batch per rank
+    weights = {k: to_dev(v) for k, v in wl.make_weights(w).items()}
     nb = w.steps if w.steps > 1 else 2
     batches = []
     for s in range(nb):
