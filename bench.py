@@ -431,7 +431,6 @@ def main():
                           logits=batches[j].get("logits")) for j in idx]
             groups.append(moe.capture_concurrent(layers, calls))
             group_batches.append(idx)
-        steps = (steps + conc - 1) // conc * conc  # whole groups
 
     def run_group(g):
         groups[g % len(groups)].replay()
@@ -456,9 +455,11 @@ def main():
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    if conc > 1:
+    if conc > 1:  # exactly `steps` steps: whole groups, then single batches
         for g in range(steps // conc):
             run_group(g)
+        for i in range(steps % conc):
+            run_step(i)
     else:
         for i in range(steps):
             run_step(i)
