@@ -61,6 +61,18 @@ MUTANTS = {
     "bwd_gate_wrong_operand": (
         "acc += (double)dlogits[(int64_t)t * E + e] * load_elem(x, dtype, (int64_t)t * d + c);",
         "acc += (double)dlogits[(int64_t)t * E + e] * load_elem(Wg, dtype, (int64_t)e * d + c);"),
+    "bwd_relu_mask_at_zero": ("if (load_elem(H, dtype, (int64_t)r * F + f) > 0.0)",
+                              "if (load_elem(H, dtype, (int64_t)r * F + f) >= 0.0)"),
+    "bwd_dw2_from_dh": ("load_elem(H, dtype, (int64_t)r * F + f);",
+                        "load_elem(dH, dtype, (int64_t)r * F + f);"),
+    "bwd_dbias_dropped": ("db[e] += dz;", "(void)dz;"),
+    "bwd_route_first_slot_only": (
+        "for (int i = 0; i < k; ++i) s += (double)w[(int64_t)t * k + i] * (double)dw[(int64_t)t * k + i];",
+        "for (int i = 0; i < 1; ++i) s += (double)w[(int64_t)t * k + i] * (double)dw[(int64_t)t * k + i];"),
+    "bwd_gate_dx_overwritten": ("double acc = load_elem(dx, dtype, (int64_t)t * d + c);",
+                                "double acc = 0.0;"),
+    "bwd_dw_token_row": ("dot += g * load_elem(Yp, dtype, (int64_t)row * d + o);",
+                         "dot += g * load_elem(Yp, dtype, (int64_t)t * d + o);"),
     "forecast_column_sum": ("a += q[i] * (double)C[(int64_t)i * E + h];",
                             "a += q[i] * (double)C[(int64_t)h * E + i];"),
 }
