@@ -73,6 +73,8 @@ MUTANTS = {
                                 "double acc = 0.0;"),
     "bwd_dw_token_row": ("dot += g * load_elem(Yp, dtype, (int64_t)row * d + o);",
                          "dot += g * load_elem(Yp, dtype, (int64_t)t * d + o);"),
+    "combine_dropped_slot_read": ("            if (row < 0) continue;\n            double wj",
+                                  "            if (row < 0) row = 0;\n            double wj"),
     "forecast_column_sum": ("a += q[i] * (double)C[(int64_t)i * E + h];",
                             "a += q[i] * (double)C[(int64_t)h * E + i];"),
 }
