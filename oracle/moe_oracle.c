@@ -120,13 +120,24 @@ void oracle_gate(const void* x, const void* Wg, int dtype, int T, int d, int E,
 
 /* ----------------------------------------------------------- route (a1) ---- */
 
+/* Strict order of routing keys: a NaN ranks above every number (and no NaN
+ * above another NaN), numbers by value (+0 and -0 equal).  The pages assume
+ * finite scores; this reading gives a diverged row (NaN logits) a defined
+ * top-k of valid expert indices, and its weights come out NaN. */
+static int ranks_above(float a, float b) {
+    if (isnan(b)) return 0;
+    if (isnan(a)) return 1;
+    return a > b;
+}
+
 /* Gate routing with expert capacity.
  *
  * [Pop-2.1.2] top-k selection; [MPMC] softmax router; [Survey-5] GShard expert
  * capacity.  Steps, in order:
  *  1. z[t][e] = logits[t][e] + bias[e], one fp32 addition.
  *  2. k times, pick the not-yet-chosen expert with the largest z; on equal z
- *     the lower expert index wins (strict '>' while scanning e upward).
+ *     the lower expert index wins (strict '>' while scanning e upward).  A NaN
+ *     z counts as larger than every number (ranks_above).
  *     Softmax is strictly increasing, so this is the top-k of the softmax.
  *  3. The k chosen softmax probabilities renormalised to sum to one:
  *     w_j = exp(z_j - z_0) / sum_i exp(z_i - z_0)  (the full softmax
@@ -162,7 +173,7 @@ int oracle_route(const float* logits, const float* bias, int T, int E, int k,
             int best = -1;
             for (int e = 0; e < E; ++e) {
                 if (taken[e]) continue;
-                if (best < 0 || z[e] > z[best]) best = e;
+                if (best < 0 || ranks_above(z[e], z[best])) best = e;
             }
             taken[best] = 1;
             ids[(int64_t)t * k + j] = best;

@@ -14,8 +14,11 @@ from conftest import ROOT
 SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
 
 MUTANTS = {
-    "tie_to_higher_index": ("if (best < 0 || z[e] > z[best]) best = e;",
-                            "if (best < 0 || z[e] >= z[best]) best = e;"),
+    "tie_to_higher_index": ("if (best < 0 || ranks_above(z[e], z[best])) best = e;",
+                            "if (best < 0 || !ranks_above(z[best], z[e])) best = e;"),
+    "nan_not_ranked_first": ("    if (isnan(a)) return 1;", "    if (isnan(a)) return 0;"),
+    "nan_compared_as_number": ("    if (isnan(b)) return 0;\n    if (isnan(a)) return 1;\n",
+                               ""),
     "weights_not_shifted": ("(float)(exp((double)z[ids[(int64_t)t * k + j]] - zmax) / denom)",
                             "(float)(exp((double)z[ids[(int64_t)t * k + j]]) / denom)"),
     "capacity_off_by_one": ("if (capacity <= 0 || p < capacity) {",

@@ -107,6 +107,45 @@ def test_route_topk_brute_force(seed):
         assert sorted(order) == list(best)
 
 
+def _nan_bits(bits):
+    return np.array([bits], np.uint32).view(np.float32)[0]
+
+
+def test_route_nan_ranks_above_every_number_hand_worked():
+    # Reading for non-finite scores (the pages assume finite ones): a NaN key
+    # ranks above every number, NaNs among themselves by index; the weights of
+    # a row whose first choice is NaN are NaN.
+    nan, inf = np.float32(np.nan), np.float32(np.inf)
+    neg_nan, ones_nan = _nan_bits(0xFFC00000), _nan_bits(0xFFFFFFFF)
+    lg = np.array([[1.0, nan, 2.0, nan, -inf],        # -> 1, 3, 2
+                   [nan, nan, nan, nan, nan],          # -> 0, 1, 2
+                   [inf, 0.0, neg_nan, -1.0, 3.0],     # -> 2, 0, 4
+                   [-inf, ones_nan, -inf, 5.0, -inf],  # -> 1, 3, 0
+                   [0.5, -0.5, 2.0, 1.0, -inf]],       # -> 2, 3, 0 (no NaN)
+                  np.float32)
+    r = oracle.route(lg, None, 3)
+    assert r["ids"].tolist() == [[1, 3, 2], [0, 1, 2], [2, 0, 4], [1, 3, 0], [2, 3, 0]]
+    assert np.isnan(r["w"][:4]).all()
+    assert np.isfinite(r["w"][4]).all()
+    assert r["counts"].tolist() == [4, 3, 4, 3, 1]
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_route_nan_and_infinities_brute_force(seed):
+    rng = np.random.default_rng(900 + seed)
+    T, E = 64, int(rng.integers(3, 12))
+    k = int(rng.integers(1, E + 1))
+    pool = np.array([np.nan, _nan_bits(0xFFC00001), np.inf, -np.inf, 0.0, -0.0, 1.0, -2.0, 2.0],
+                    np.float32)
+    lg = pool[rng.integers(0, len(pool), (T, E))]
+    r = oracle.route(lg, None, k)
+    for t in range(T):
+        z = lg[t]
+        order = sorted(range(E), key=lambda e: (0, 0.0, e) if np.isnan(z[e])
+                       else (1, -float(z[e]), e))[:k]
+        assert r["ids"][t].tolist() == order
+
+
 @pytest.mark.parametrize("seed", range(4))
 def test_route_weights_are_renormalised_full_softmax(seed):
     rng = np.random.default_rng(200 + seed)
