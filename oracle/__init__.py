@@ -20,6 +20,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+# the same source built with -fopenmp: its independent token / row loops run on
+# all host cores (every value computed by the same operations in the same order)
+_LIB_OMP = os.path.join(_HERE, "liboracle_omp.so")
 
 F32 = 0
 BF16 = 1
@@ -29,15 +32,28 @@ _lib = None
 _lib_path = os.environ.get("MOE_ORACLE_LIB") or _LIB
 
 
-def build(force: bool = False) -> str:
-    """Compile moe_oracle.c into liboracle.so (no fused multiply-add, no fast math)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
+def build(force: bool = False, parallel: bool = False) -> str:
+    """Compile moe_oracle.c into liboracle.so (no fused multiply-add, no fast
+    math), or with ``parallel`` into liboracle_omp.so (the same flags plus
+    -fopenmp)."""
+    out = _LIB_OMP if parallel else _LIB
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
+        tmp = out + f".tmp{os.getpid()}"
         subprocess.check_call(
             ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
-             "-shared", "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+             *(["-fopenmp"] if parallel else []), "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, out)
+    return out
+
+
+def use_parallel(parallel: bool = True, threads: int = 0) -> int:
+    """Switch the wrappers to the OpenMP build (or back); returns the thread
+    count the marked loops use (``threads`` > 0 caps it)."""
+    use_library(build(parallel=True) if parallel else None)
+    lib = _load()
+    if threads > 0:
+        lib.oracle_set_threads(int(threads))
+    return int(lib.oracle_threads())
 
 
 def use_library(path: str | None) -> None:
@@ -54,6 +70,8 @@ def _load():
     if _lib is None:
         if _lib_path == _LIB:
             build()
+        elif _lib_path == _LIB_OMP:
+            build(parallel=True)
         lib = ctypes.CDLL(_lib_path)
         p, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
         lib.oracle_gate.argtypes = [p, p, i32, i32, i32, i32, p]
@@ -87,6 +105,12 @@ def _load():
         lib.oracle_route_backward.restype = None
         lib.oracle_gate_backward.argtypes = [p, p, i32, i32, i32, i32, p, p, p]
         lib.oracle_gate_backward.restype = None
+        lib.oracle_expert_ffn_rows.argtypes = [p, p, i32, p, p, i32, i32, i32, p, p]
+        lib.oracle_expert_ffn_rows.restype = None
+        lib.oracle_threads.argtypes = []
+        lib.oracle_threads.restype = i32
+        lib.oracle_set_threads.argtypes = [i32]
+        lib.oracle_set_threads.restype = None
         lib.oracle_round_bf16.argtypes = [ctypes.c_double]
         lib.oracle_round_bf16.restype = ctypes.c_uint16
         _lib = lib
@@ -189,15 +213,12 @@ def expert_ffn_rows(rows: np.ndarray, experts, W1: np.ndarray, W2: np.ndarray,
     dt = _dtype_code(rows)
     E, F, d = W1.shape
     n = rows.shape[0]
+    ex = _c(np.asarray(experts), np.int32)
+    assert ex.shape == (n,) and (n == 0 or (ex.min() >= 0 and ex.max() < E))
     Y = np.empty((n, d), rows.dtype)
     H = np.empty((n, F), rows.dtype) if want_h else None
-    lib = _load()
-    es = rows.itemsize
-    for i, e in enumerate(np.asarray(experts).tolist()):
-        hp = None if H is None else ctypes.c_void_p(H.ctypes.data + i * F * es)
-        lib.oracle_expert_ffn_row(ctypes.c_void_p(rows.ctypes.data + i * d * es), _ptr(W1),
-                                  _ptr(W2), dt, int(e), d, F, hp,
-                                  ctypes.c_void_p(Y.ctypes.data + i * d * es))
+    _load().oracle_expert_ffn_rows(_ptr(rows), _ptr(ex), n, _ptr(W1), _ptr(W2), dt, d, F,
+                                   _ptr(H), _ptr(Y))
     return (Y, H) if want_h else Y
 
 

@@ -43,9 +43,17 @@
  * to the storage type (bf16 or fp32) of the tensor it writes.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC.
+ * A second build adds -fopenmp: the loops over tokens and rows marked
+ * "omp parallel for" below are independent (each iteration writes its own
+ * output row and reads nothing another iteration writes), so the threaded
+ * build computes every value with the same operations in the same order as
+ * the single-threaded one; only which core computes a row changes.
  */
 #include <math.h>
 #include <stdint.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 #include <stdlib.h>
 #include <string.h>
 
@@ -100,6 +108,22 @@ static size_t elem_size(int dtype) { return dtype == ORC_BF16 ? 2u : 4u; }
 /* Exposed so the tests can pin the rounding against numpy's float32 path. */
 uint16_t oracle_round_bf16(double v) { return double_to_bf16_bits(v); }
 
+/* Threads the marked loops may use (1 in the single-threaded build). */
+int oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------ gate (a0) ---- */
 
 /* Router logits of each token: logits[t][e] = sum_c x[t][c] * Wg[e][c].
@@ -108,6 +132,7 @@ uint16_t oracle_round_bf16(double v) { return double_to_bf16_bits(v); }
  * double over c ascending, rounded once to fp32. */
 void oracle_gate(const void* x, const void* Wg, int dtype, int T, int d, int E,
                  float* logits) {
+#pragma omp parallel for schedule(static)
     for (int t = 0; t < T; ++t)
         for (int e = 0; e < E; ++e) {
             double acc = 0.0;
@@ -229,6 +254,7 @@ void oracle_dispatch(const void* x, int dtype, int T, int d, int k,
                      const int32_t* row_slot, int R, void* Xp) {
     size_t rowbytes = elem_size(dtype) * (size_t)d;
     (void)T;
+#pragma omp parallel for schedule(static)
     for (int row = 0; row < R; ++row) {
         int t = row_slot[row] / k;
         memcpy((char*)Xp + (size_t)row * rowbytes, (const char*)x + (size_t)t * rowbytes,
@@ -271,15 +297,35 @@ void oracle_expert_ffn_row(const void* xrow, const void* W1, const void* W2,
 }
 
 /* Expert computation over all groups: rows [offsets[e], offsets[e+1]) go
- * through expert e.  H may be NULL. */
+ * through expert e, i.e. row r goes through the e with
+ * offsets[e] <= r < offsets[e+1] (the last e with offsets[e] <= r, so empty
+ * groups are skipped).  H may be NULL. */
 void oracle_expert_ffn(const void* Xp, const void* W1, const void* W2, int dtype,
                        int E, int d, int F, const int32_t* offsets, void* H, void* Yp) {
     size_t es = elem_size(dtype);
-    for (int e = 0; e < E; ++e)
-        for (int row = offsets[e]; row < offsets[e + 1]; ++row)
-            oracle_expert_ffn_row((const char*)Xp + (size_t)row * d * es, W1, W2, dtype, e, d, F,
-                                  H ? (char*)H + (size_t)row * F * es : NULL,
-                                  (char*)Yp + (size_t)row * d * es);
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int row = offsets[0]; row < offsets[E]; ++row) {
+        int lo = 0, hi = E - 1;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) / 2;
+            if (offsets[mid] <= row) lo = mid; else hi = mid - 1;
+        }
+        oracle_expert_ffn_row((const char*)Xp + (size_t)row * d * es, W1, W2, dtype, lo, d, F,
+                              H ? (char*)H + (size_t)row * F * es : NULL,
+                              (char*)Yp + (size_t)row * d * es);
+    }
+}
+
+/* Selected rows, each through its own expert: rows[i] through experts[i]
+ * (the full-size parity checks sample rows this way).  H may be NULL. */
+void oracle_expert_ffn_rows(const void* rows, const int32_t* experts, int n, const void* W1,
+                            const void* W2, int dtype, int d, int F, void* H, void* Y) {
+    size_t es = elem_size(dtype);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n; ++i)
+        oracle_expert_ffn_row((const char*)rows + (size_t)i * d * es, W1, W2, dtype, experts[i],
+                              d, F, H ? (char*)H + (size_t)i * F * es : NULL,
+                              (char*)Y + (size_t)i * d * es);
 }
 
 /* --------------------------------------------------------- combine (a4) ---- */
@@ -291,19 +337,24 @@ void oracle_expert_ffn(const void* Xp, const void* W1, const void* W2, int dtype
  * token with no kept slot gets zeros. */
 void oracle_combine(const void* Yp, int dtype, int T, int d, int k,
                     const int32_t* slot_row, const float* w, void* y) {
-    double* acc = (double*)malloc(sizeof(double) * (size_t)d);
-    if (!acc) return;
-    for (int t = 0; t < T; ++t) {
-        for (int o = 0; o < d; ++o) acc[o] = 0.0;
-        for (int j = 0; j < k; ++j) {
-            int32_t row = slot_row[(int64_t)t * k + j];
-            if (row < 0) continue;
-            double wj = (double)w[(int64_t)t * k + j];
-            for (int o = 0; o < d; ++o) acc[o] += wj * load_elem(Yp, dtype, (int64_t)row * d + o);
+#pragma omp parallel
+    {
+        double* acc = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(static)
+        for (int t = 0; t < T; ++t) {
+            if (!acc) continue;
+            for (int o = 0; o < d; ++o) acc[o] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int32_t row = slot_row[(int64_t)t * k + j];
+                if (row < 0) continue;
+                double wj = (double)w[(int64_t)t * k + j];
+                for (int o = 0; o < d; ++o)
+                    acc[o] += wj * load_elem(Yp, dtype, (int64_t)row * d + o);
+            }
+            for (int o = 0; o < d; ++o) store_elem(y, dtype, (int64_t)t * d + o, acc[o]);
         }
-        for (int o = 0; o < d; ++o) store_elem(y, dtype, (int64_t)t * d + o, acc[o]);
+        free(acc);
     }
-    free(acc);
 }
 
 /* ------------------------------------------------------ popularity (a5) ---- */

@@ -5,9 +5,12 @@ it holds none of the layer's arithmetic (no routing, no FFN, no combine).
 Both the CUDA library and the CPU oracle receive the arrays built here.
 
 Generator: numpy PCG64, seed = 1000 * workload + 10 * step + tensor_id
-(+ 100000 * rank for independent per-rank batches).  Floats are drawn in
-fp32; bf16 tensors are rounded to bf16 once here (nearest even) and travel as
-uint16 bit patterns, so both sides read the same bits.
+(+ 100000 * rank for independent per-rank batches).  The expert weight stacks
+W1 and W2 draw expert e's slice from its own stream, PCG64 seeded with
+SeedSequence(seed, spawn_key=(e,)), so the experts are drawn in parallel
+threads.  Floats are drawn in fp32; bf16 tensors are rounded to bf16 once here
+(nearest even) and travel as uint16 bit patterns, so both sides read the same
+bits.
 
 Workloads (sizes from the pages' MoE settings; expert FFN is FC-ReLU-FC as in
 PopFetcher, section 5.1; top-k gating with GShard capacity as in "A Survey on
@@ -22,8 +25,10 @@ Mixture of Experts", section 5):
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 from fractions import Fraction
 
 import numpy as np
@@ -79,9 +84,12 @@ WORKLOADS = {
 BW_SWEEP_TOKENS = (8192, 16384, 32768, 65536)
 
 
+def seed_for(w: Workload, step: int, tensor_id: int, rank: int = 0) -> int:
+    return 1000 * w.index + 10 * step + tensor_id + 100000 * rank
+
+
 def rng_for(w: Workload, step: int, tensor_id: int, rank: int = 0) -> np.random.Generator:
-    return np.random.Generator(np.random.PCG64(1000 * w.index + 10 * step + tensor_id
-                                               + 100000 * rank))
+    return np.random.Generator(np.random.PCG64(seed_for(w, step, tensor_id, rank)))
 
 
 # ------------------------------------------------------------ bf16 storage --
@@ -103,11 +111,19 @@ def _normal(rng, shape, scale, dtype):
     return to_bf16_bits(a) if dtype == "bf16" else a
 
 
-def _normal_chunked(rng, E, rows, cols, scale, dtype):
-    """[E, rows, cols] drawn expert by expert to bound host memory."""
+def _normal_experts(seed, E, rows, cols, scale, dtype):
+    """[E, rows, cols]: expert e from PCG64(SeedSequence(seed, spawn_key=(e,))),
+    the experts drawn in parallel threads (numpy releases the GIL while it
+    fills large arrays)."""
     out = np.empty((E, rows, cols), np.uint16 if dtype == "bf16" else np.float32)
-    for e in range(E):
+
+    def one(e):
+        rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=(e,))))
         out[e] = _normal(rng, (rows, cols), scale, dtype)
+
+    workers = max(1, min(E, os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
+        list(ex.map(one, range(E)))
     return out
 
 
@@ -142,9 +158,9 @@ def make_weights(w: Workload, rank: int = 0) -> dict:
         out["Wg"] = _normal(rng_for(w, 0, TENSOR_WG, rank), (w.E, w.d), 1.0 / math.sqrt(w.d),
                             w.dtype)
     if not w.identity_experts:
-        out["W1"] = _normal_chunked(rng_for(w, 0, TENSOR_W1, rank), w.E, w.F, w.d,
+        out["W1"] = _normal_experts(seed_for(w, 0, TENSOR_W1, rank), w.E, w.F, w.d,
                                     1.0 / math.sqrt(w.d), w.dtype)
-        out["W2"] = _normal_chunked(rng_for(w, 0, TENSOR_W2, rank), w.E, w.d, w.F,
+        out["W2"] = _normal_experts(seed_for(w, 0, TENSOR_W2, rank), w.E, w.d, w.F,
                                     1.0 / math.sqrt(w.F), w.dtype)
     return out
 

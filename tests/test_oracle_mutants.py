@@ -76,15 +76,23 @@ MUTANTS = {
                                 "double acc = 0.0;"),
     "bwd_dw_token_row": ("dot += g * load_elem(Yp, dtype, (int64_t)row * d + o);",
                          "dot += g * load_elem(Yp, dtype, (int64_t)t * d + o);"),
-    "combine_dropped_slot_read": ("            if (row < 0) continue;\n            double wj",
-                                  "            if (row < 0) row = 0;\n            double wj"),
+    "combine_dropped_slot_read": ("                if (row < 0) continue;\n                double wj",
+                                  "                if (row < 0) row = 0;\n                double wj"),
     "forecast_column_sum": ("a += q[i] * (double)C[(int64_t)i * E + h];",
                             "a += q[i] * (double)C[(int64_t)h * E + i];"),
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_reject_mutant(name, tmp_path):
+# Mutants inside the loops the OpenMP build runs in parallel, planted again in
+# that build (the pins then run on four threads).
+PARALLEL_LOOP_MUTANTS = ["w1_transposed", "relu_missing", "h_not_rounded", "w2_wrong_expert",
+                         "combine_first_weight_only", "combine_dropped_slot_read",
+                         "dispatch_wrong_token", "gate_transposed"]
+CASES = [(n, False) for n in sorted(MUTANTS)] + [(n, True) for n in PARALLEL_LOOP_MUTANTS]
+
+
+@pytest.mark.parametrize("name,parallel", CASES)
+def test_pins_reject_mutant(name, parallel, tmp_path):
     old, new = MUTANTS[name]
     src = open(SRC).read()
     assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
@@ -92,8 +100,9 @@ def test_pins_reject_mutant(name, tmp_path):
     mutated.write_text(src.replace(old, new))
     lib = tmp_path / "liboracle_mutant.so"
     subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
-                           "-fPIC", "-shared", "-o", str(lib), str(mutated), "-lm"])
-    env = dict(os.environ, MOE_ORACLE_LIB=str(lib))
+                           "-fPIC", *(["-fopenmp"] if parallel else []), "-shared", "-o",
+                           str(lib), str(mutated), "-lm"])
+    env = dict(os.environ, MOE_ORACLE_LIB=str(lib), OMP_NUM_THREADS="4")
     res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                           os.path.join(ROOT, "tests", "test_oracle_pins.py"),
                           os.path.join(ROOT, "tests", "test_oracle_backward.py")],

@@ -66,3 +66,17 @@ def test_backward_generators_are_seeded_and_shaped():
     lg = wl.router_logits(w)
     assert lg.dtype == np.float32 and lg.shape == (64, w.E)
     assert np.array_equal(lg, wl.router_logits(w))
+
+
+def test_expert_weights_come_from_per_expert_streams():
+    # expert e's slice is drawn from PCG64(SeedSequence(seed, spawn_key=(e,))),
+    # whatever thread draws it
+    w = wl.tiny("c", T=8, d=16, E=5, k=2, F=24)
+    W = wl.make_weights(w)
+    seed = wl.seed_for(w, 0, wl.TENSOR_W1)
+    for e in range(w.E):
+        rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=(e,))))
+        ref = wl.to_bf16_bits(rng.standard_normal((24, 16), dtype=np.float32)
+                              * np.float32(1 / math.sqrt(16)))
+        assert np.array_equal(W["W1"][e], ref), e
+    assert not np.array_equal(W["W1"][0], W["W1"][1])
