@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
 #include <utility>
 
 #include "../../include/moe.h"
@@ -43,34 +45,51 @@ inline int current_device() {
     return dev;
 }
 
-// SM count of the current device (queried once per device).
+// SM count of the current device (queried once per device; host threads that
+// race on the first query store the same value).
 inline int num_sms() {
-    static int cache[kMaxDevices] = {};
+    static std::atomic<int> cache[kMaxDevices] = {};
     const int dev = current_device();
     if (dev < 0) return 148;
-    if (cache[dev] == 0) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_acquire);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
-        cache[dev] = n;
+        cache[dev].store(n, std::memory_order_release);
     }
-    return cache[dev];
+    return n;
 }
+
+#ifdef MOE_TEST_HOOKS
+// Test builds only: a cap on the persistent GEMMs' CTA count (abi.cu), so that
+// a small problem makes one CTA (or one pair) walk many tiles.
+int test_max_ctas();
+inline int test_cap(int grid) {
+    const int c = test_max_ctas();
+    return (c > 0 && grid > c) ? c : grid;
+}
+#else
+inline int test_cap(int grid) { return grid; }
+#endif
 
 // Raises a kernel's dynamic shared-memory limit once per device (and again only
 // if a larger size is needed), so launches inside a stream capture make no
-// attribute calls.  One static cache per kernel (the kernel is the template
-// argument, so kernels that share a signature do not share a cache).
+// attribute calls.  One cache per kernel (the kernel is the template argument,
+// so kernels that share a signature do not share a cache); raising the limit
+// is serialised so that a smaller request never undoes a larger one.
 template <auto kern>
 inline int ensure_smem(int bytes) {
-    static int done[kMaxDevices] = {};
+    static std::atomic<int> done[kMaxDevices] = {};
+    static std::mutex mu;
     const int dev = current_device();
     if (dev < 0) return MOE_ERR_CUDA;
-    if (done[dev] >= bytes) return MOE_OK;
+    if (done[dev].load(std::memory_order_acquire) >= bytes) return MOE_OK;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev].load(std::memory_order_relaxed) >= bytes) return MOE_OK;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
-    done[dev] = bytes;
+    done[dev].store(bytes, std::memory_order_release);
     return MOE_OK;
 }
 

@@ -201,7 +201,8 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
             uint32_t phase = 0;
             long long issued = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            const int first = test_stall() ? total : blockIdx.x;
+            for (int tile = first; ok && tile < total; tile += gridDim.x) {
                 int e, m0, rows, n0, k0, nk, kr;
                 coord(tile, e, m0, rows, n0, k0, nk, kr);
                 for (int b = 0; b < planes * nk; ++b) {
@@ -454,7 +455,7 @@ int launch_bwd(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
                const BwdArgs& args, long long ub, cudaStream_t st) {
     const int smem = fixed_bytes<EPI>() + 4 * (args.E + 1);
     if (ensure_smem<gemm_bwd_kernel<A_MN, KVAR, EPI>>(smem) != MOE_OK) return MOE_ERR_CUDA;
-    const int grid = (int)(ub < num_sms() ? ub : num_sms());
+    const int grid = test_cap((int)(ub < num_sms() ? ub : num_sms()));
     if (grid <= 0) return MOE_OK;
     return launch_pdl(gemm_bwd_kernel<A_MN, KVAR, EPI>, grid, kThreads, smem, st, ta, tb, tc_map,
                       args, device_error_word());
@@ -480,6 +481,10 @@ inline BwdArgs grouped(void* C, const void* Hmask, int M_fix, int N, int K_fix, 
 
 }  // namespace bwd
 }  // namespace tc
+
+#ifdef MOE_TEST_HOOKS
+int test_stall_bwd(int v) { return tc::set_test_stall(v); }
+#endif
 
 // dH = (dYp . W2_e) * [H > 0] and dXp = dH . W1_e over the grouped rows, then
 // dW2 = dYp_e^T H_e and dW1 = dH_e^T Xp_e per expert (fp32).

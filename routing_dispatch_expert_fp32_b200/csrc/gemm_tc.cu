@@ -45,6 +45,12 @@ namespace tc {
 #define MOE_PAIR_MIN_ROWS_PER_GROUP 1024
 #endif
 constexpr long long kPairMinRowsPerGroup = MOE_PAIR_MIN_ROWS_PER_GROUP;
+// Dense groups: pair tiles for whole 256-row blocks plus 1-CTA tiles for the
+// tails (0: pair tiles for everything).
+#ifndef MOE_SPLIT_TAILS
+#define MOE_SPLIT_TAILS 0
+#endif
+constexpr bool kSplitTails = MOE_SPLIT_TAILS != 0;
 
 template <int BN>
 struct Cfg {
@@ -85,7 +91,7 @@ template <int BN_MAX, bool RELU, typename TOut, int MODE = MODE_PLAIN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                TOut* __restrict__ C, int N, int K, int E, const int32_t* __restrict__ offsets,
-               int single_M, int R_max, Gather gat, int32_t* err) {
+               int single_M, int R_max, Gather gat, int part, int32_t* err) {
     using G = Cfg<BN_MAX>;
     constexpr int S = G::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -125,7 +131,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     }
     pdl_wait();  // everything above touched only this CTA's on-chip state
     pdl_trigger();
-    const int mtiles = build_tile_table(offsets, single_M, E, 1, BM, R_max, s_prefix, s_warp, err);
+    const int mtiles =
+        build_tile_table(offsets, single_M, E, 1, BM, R_max, s_prefix, s_warp, err, part);
     constexpr int bn = BN_MAX;
     const int nt = (N + bn - 1) / bn;
     const int total = mtiles * nt;
@@ -149,8 +156,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         long long issued = 0;
         bool ok = true;
         const int n_slots = gat.T * gat.k;
-        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-            const TileCoord c = tile_coord(tile, s_prefix, E, offsets, single_M, BM, bn, nt);
+        const int first = test_stall() ? total : blockIdx.x;
+        for (int tile = first; ok && tile < total; tile += gridDim.x) {
+            const TileCoord c = tile_coord(tile, s_prefix, E, offsets, single_M, BM, bn, nt, part);
             const int b_row = c.e * N + c.n0;
             int xr[4];
 #pragma unroll
@@ -199,8 +207,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
             uint32_t phase = 0;
             long long issued = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const TileCoord c = tile_coord(tile, s_prefix, E, offsets, single_M, BM, bn, nt);
+            const int first = test_stall() ? total : blockIdx.x;
+            for (int tile = first; ok && tile < total; tile += gridDim.x) {
+                const TileCoord c = tile_coord(tile, s_prefix, E, offsets, single_M, BM, bn, nt, part);
                 const int b_row = c.e * N + c.n0;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, err)) {
@@ -268,7 +277,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
         int it = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-            const TileCoord c = tile_coord(tile, s_prefix, E, offsets, single_M, BM, bn, nt);
+            const TileCoord c = tile_coord(tile, s_prefix, E, offsets, single_M, BM, bn, nt, part);
             const int acc = it & 1;
             if (!mbar_wait(tfull + acc, (it >> 1) & 1, abort_flag, err)) break;
             tc_fence_after();
@@ -389,7 +398,7 @@ template <bool RELU>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b, __nv_bfloat16* __restrict__ C, int N,
-                int K, int E, const int32_t* __restrict__ offsets, int R_max, int32_t* err) {
+                int K, int E, const int32_t* __restrict__ offsets, int R_max, int part, int32_t* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~static_cast<uintptr_t>(1023u));
@@ -430,7 +439,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
     pdl_wait();  // everything above touched only this CTA's on-chip state
     pdl_trigger();
     const int pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-    const int mtiles = build_tile_table(offsets, 0, E, 1, BM, R_max, s_prefix, s_warp, err);
+    const int mtiles = build_tile_table(offsets, 0, E, 1, BM, R_max, s_prefix, s_warp, err, part);
     constexpr int bn = BN;
     const int nt = (N + bn - 1) / bn;
     const int total = mtiles * nt;
@@ -452,8 +461,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
             uint32_t phase = 0;
             long long issued = 0;
             bool ok = true;
-            for (int tile = pair_id; ok && tile < total; tile += npairs) {
-                const TileCoord c = tile_coord(tile, s_prefix, E, offsets, 0, BM, bn, nt);
+            const int first = test_stall() ? total : pair_id;
+            for (int tile = first; ok && tile < total; tile += npairs) {
+                const TileCoord c = tile_coord(tile, s_prefix, E, offsets, 0, BM, bn, nt, part);
                 const int a_row = c.row0 + HALF * (int)rank;
                 const int b_row = c.e * N + c.n0 + b_half * (int)rank;
                 for (int kb = 0; kb < nk; ++kb) {
@@ -530,7 +540,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
         int it = 0;
         for (int tile = pair_id; tile < total; tile += npairs, ++it) {
-            const TileCoord c = tile_coord(tile, s_prefix, E, offsets, 0, BM, bn, nt);
+            const TileCoord c = tile_coord(tile, s_prefix, E, offsets, 0, BM, bn, nt, part);
             const int acc = it & 1;
             if (!mbar_wait(tfull + acc, (it >> 1) & 1, abort_flag, err)) break;
             tc_fence_after();
@@ -566,7 +576,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
 template <int BN, bool RELU, typename TOut, int MODE = MODE_PLAIN>
 static int launch(const void* A, const void* B, TOut* C, int N, int K, int E,
                   const int32_t* offsets, int single_M, int R_max, cudaStream_t st,
-                  Gather gat = Gather{nullptr, nullptr, 1, 0}) {
+                  Gather gat = Gather{nullptr, nullptr, 1, 0}, int part = PART_ALL) {
     using G = Cfg<BN>;
     if (R_max <= 0 || N <= 0) return MOE_OK;
     CUtensorMap ta, tb;
@@ -580,15 +590,17 @@ static int launch(const void* A, const void* B, TOut* C, int N, int K, int E,
     auto kern = gemm_tc_kernel<BN, RELU, TOut, MODE>;
     if (ensure_smem<gemm_tc_kernel<BN, RELU, TOut, MODE>>(smem) != MOE_OK) return MOE_ERR_CUDA;
     const int nt = (N + BN - 1) / BN;
-    const long long ub = ((long long)R_max / BM + E) * nt;
-    const int grid = (int)(ub < num_sms() ? ub : num_sms());
+    // tiles, upper bound (a tail part has at most kSplitRows / BM tiles per group)
+    const long long ub = part == PART_TAIL ? (long long)E * (kSplitRows / BM) * nt
+                                           : ((long long)R_max / BM + E) * nt;
+    const int grid = test_cap((int)(ub < num_sms() ? ub : num_sms()));
     return launch_pdl(kern, grid, kThreads, smem, st, ta, tb, C, N, K, E, offsets, single_M, R_max,
-                      gat, device_error_word());
+                      gat, part, device_error_word());
 }
 
 template <bool RELU>
 static int launch_pair(const void* A, const void* B, __nv_bfloat16* C, int N, int K, int E,
-                       const int32_t* offsets, int R_max, cudaStream_t st) {
+                       const int32_t* offsets, int R_max, cudaStream_t st, int part = PART_ALL) {
     if (R_max <= 0 || N <= 0) return MOE_OK;
     CUtensorMap ta, tb;
     if (make_tmap(&ta, A, K, R_max, pair::HALF) != MOE_OK) return MOE_ERR_CUDA;
@@ -599,12 +611,17 @@ static int launch_pair(const void* A, const void* B, __nv_bfloat16* C, int N, in
     const int nt = (N + pair::BN - 1) / pair::BN;
     const long long ub = ((long long)R_max / pair::BM + E) * nt;  // pair tiles, upper bound
     const int pairs_max = num_sms() / 2;
-    const int pairs = (int)(ub < pairs_max ? ub : pairs_max);
+    int pairs = (int)(ub < pairs_max ? ub : pairs_max);
+    pairs = test_cap(2 * pairs) / 2 > 0 ? test_cap(2 * pairs) / 2 : 1;
     return launch_pdl(kern, 2 * pairs, kThreads, smem, st, ta, tb, C, N, K, E, offsets, R_max,
-                      device_error_word());
+                      part, device_error_word());
 }
 
 }  // namespace tc
+
+#ifdef MOE_TEST_HOOKS
+int test_stall_tc(int v) { return tc::set_test_stall(v); }
+#endif
 
 int launch_gemm_tc_bf16(const void* A, const void* B, void* C, bool out_f32, int N, int K, int E,
                         const int32_t* offsets, int single_M, int R_max, bool relu,
@@ -626,8 +643,21 @@ int launch_gemm_tc_bf16(const void* A, const void* B, void* C, bool out_f32, int
     // B200: the skewed_drops second GEMM, 1.2 waves, 63.2 -> 58.7 us; its first
     // GEMM, 8.6 waves, and both multistep_window GEMMs are slower with pairs).
     const long long tiles_1cta = ((long long)R_max / BM + E) * ((N + 255) / 256);
-    if (offsets != nullptr && ((long long)R_max >= (long long)kPairMinRowsPerGroup * E ||
-                               tiles_1cta < 3LL * num_sms())) {
+    const bool dense = (long long)R_max >= (long long)kPairMinRowsPerGroup * E;
+    if (offsets != nullptr && dense && kSplitTails) {
+        // whole 256-row blocks of every group on pair tiles, then the rows
+        // after them on 128-row tiles: a group pads to 128 rows, not 256
+        int rc = relu ? launch_pair<true>(A, B, Cb, N, K, E, offsets, R_max, st, PART_BLOCKS)
+                      : launch_pair<false>(A, B, Cb, N, K, E, offsets, R_max, st, PART_BLOCKS);
+        if (rc != MOE_OK) return rc;
+        const Gather none{nullptr, nullptr, 1, 0};
+        if (relu)
+            return launch<256, true, __nv_bfloat16>(A, B, Cb, N, K, E, offsets, 0, R_max, st, none,
+                                                     PART_TAIL);
+        return launch<256, false, __nv_bfloat16>(A, B, Cb, N, K, E, offsets, 0, R_max, st, none,
+                                                  PART_TAIL);
+    }
+    if (offsets != nullptr && (dense || tiles_1cta < 3LL * num_sms())) {
         if (relu) return launch_pair<true>(A, B, Cb, N, K, E, offsets, R_max, st);
         return launch_pair<false>(A, B, Cb, N, K, E, offsets, R_max, st);
     }

@@ -26,6 +26,29 @@ __device__ __forceinline__ int group_off(const int32_t* __restrict__ offsets, in
     return offsets ? offsets[e] : (e == 0 ? 0 : single_M);
 }
 
+// Which rows of each group a launch covers: all of them (PART_ALL), the whole
+// kSplitRows-row blocks from the group's start (PART_BLOCKS), or the rows after
+// the last whole block (PART_TAIL).  A dense grouped GEMM runs the blocks on
+// 2-CTA 256-row tiles and the tails on 128-row tiles, so a group pads to 128
+// rows instead of 256.
+enum { PART_ALL = 0, PART_BLOCKS = 1, PART_TAIL = 2 };
+constexpr int kSplitRows = 256;
+
+// First row and row count of group e's part (groups with invalid bounds get no
+// tiles from build_tile_table, so tile_coord never lands on them).
+__device__ __forceinline__ void group_part(const int32_t* __restrict__ offsets, int e,
+                                           int single_M, int part, int& a, int& m) {
+    a = group_off(offsets, e, single_M);
+    m = group_off(offsets, e + 1, single_M) - a;
+    if (part == PART_BLOCKS) {
+        m = (m / kSplitRows) * kSplitRows;
+    } else if (part == PART_TAIL) {
+        const int whole = (m / kSplitRows) * kSplitRows;
+        a += whole;
+        m -= whole;
+    }
+}
+
 // Builds s_prefix[0..E] (exclusive prefix of tiles per group) with all threads
 // of the block; returns the total tile count.  Invalid offsets (negative,
 // decreasing, or beyond R_max) give that group no tiles and flag an error.
@@ -33,7 +56,7 @@ __device__ __forceinline__ int group_off(const int32_t* __restrict__ offsets, in
 // thread of the block (contains __syncthreads).
 __device__ inline int build_tile_table(const int32_t* __restrict__ offsets, int single_M, int E,
                                        int nt, int BM, int R_max, int32_t* s_prefix,
-                                       int32_t* s_warp, int32_t* err) {
+                                       int32_t* s_warp, int32_t* err, int part = PART_ALL) {
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int lane = tid & 31, wid = tid >> 5, nw = nthr >> 5;
     int carry = 0;
@@ -45,7 +68,9 @@ __device__ inline int build_tile_table(const int32_t* __restrict__ offsets, int 
             if (a < 0 || b < a || b > R_max) {
                 if (blockIdx.x == 0) flag_error(err, MOE_DEVERR_OFFSETS);
             } else {
-                tiles = ((b - a + BM - 1) / BM) * nt;
+                int pa, pm;
+                group_part(offsets, e, single_M, part, pa, pm);
+                tiles = ((pm + BM - 1) / BM) * nt;
             }
         }
         int incl = tiles;
@@ -77,19 +102,19 @@ __device__ inline int build_tile_table(const int32_t* __restrict__ offsets, int 
 }
 
 // Maps a linear tile index to its coordinates, given the prefix of M-tiles per
-// group (s_prefix from build_tile_table with nt = 1) and nt N-tiles per group:
-// group e owns tiles [nt * s_prefix[e], nt * s_prefix[e+1]).
+// group (s_prefix from build_tile_table with nt = 1 and the same part) and nt
+// N-tiles per group: group e owns tiles [nt * s_prefix[e], nt * s_prefix[e+1]).
 __device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* s_prefix, int E,
                                                 const int32_t* __restrict__ offsets, int single_M,
-                                                int BM, int BN, int nt) {
+                                                int BM, int BN, int nt, int part = PART_ALL) {
     int lo = 0, hi = E - 1;  // largest e with nt * s_prefix[e] <= tile
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (nt * s_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
     }
     const int e = lo;
-    const int a = group_off(offsets, e, single_M);
-    const int m = group_off(offsets, e + 1, single_M) - a;
+    int a, m;
+    group_part(offsets, e, single_M, part, a, m);
     const int mt = (m + BM - 1) / BM;
     const int local = tile - nt * s_prefix[e];
     const int mb = local % mt, nb = local / mt;

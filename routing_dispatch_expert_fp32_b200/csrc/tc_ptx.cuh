@@ -15,7 +15,27 @@ constexpr int BM = 128;
 constexpr int BK = 64;  // one 128-byte swizzle row of bf16
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
-constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
+// Longest wait of one pipeline barrier before the kernel gives up: 2 s (a
+// test build shortens it with -DMOE_WAIT_LIMIT_NS).
+#ifndef MOE_WAIT_LIMIT_NS
+#define MOE_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr unsigned long long kTimeoutNs = MOE_WAIT_LIMIT_NS;
+
+#ifdef MOE_TEST_HOOKS
+// Test builds only (-DMOE_TEST_HOOKS; never the shipped library): a flag of
+// this translation unit that makes the GEMM producers issue no loads at all,
+// so that the MMA and epilogue waits run out with nothing in flight.
+static __device__ int s_test_stall = 0;
+__device__ __forceinline__ bool test_stall() {
+    return *reinterpret_cast<volatile int*>(&s_test_stall) != 0;
+}
+static int set_test_stall(int v) {
+    return cudaMemcpyToSymbol(s_test_stall, &v, sizeof v) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+#else
+__device__ __forceinline__ bool test_stall() { return false; }
+#endif
 
 // ------------------------------------------------------------ PTX wrappers --
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -221,16 +241,18 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once (thread-safe static
+// initialisation; null if the driver does not provide it).
 static EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
+    static const EncodeTiledFn fn = [] {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
                                              &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return static_cast<EncodeTiledFn>(nullptr);
+    }();
     return fn;
 }
 

@@ -42,6 +42,12 @@ def run_ffn(moe, Xp, W1, W2, offsets, Rmax):
     ([0, 65, 200], 72, 100, "f32"),
     # enough 128-row tiles (>= 3 waves) that the first GEMM stays on 1-CTA tiles
     ([1000, 1, 0, 1999, 1000], 64, 4096, "bf16"),
+    # groups just under and over 16-, 64-, 128- and 256-row boundaries, K not a
+    # multiple of 64, odd and even numbers of k-blocks
+    ([1, 15, 16, 17, 63, 64, 65, 0, 255, 256, 257, 511, 513], 136, 384, "bf16"),
+    ([1, 15, 16, 17, 63, 64, 65, 0, 255, 256, 257, 511, 513], 256, 640, "bf16"),
+    ([3, 40, 0, 129, 300, 2], 192, 256, "bf16"),
+    ([70, 5, 1, 33], 384, 128, "bf16"),
 ])
 def test_ffn_small_shapes_elementwise(moe, sizes, d, F, dtype):
     E = len(sizes)
@@ -57,6 +63,27 @@ def test_ffn_small_shapes_elementwise(moe, sizes, d, F, dtype):
         tol = dict(max_abs_frac=1e-5, mean_rel=1e-6) if dtype == "f32" else {}
         assert_close(H[:R], Hr, "H", **tol)
         assert_close(Yp[:R], Yr, "Yp", **tol)
+    assert not H[R:].any() and not Yp[R:].any()
+    assert moe.moe_device_error() == 0
+
+
+@pytest.mark.parametrize("sizes,d,F", [
+    ([0, 1, 17, 255, 256, 257, 600, 16], 256, 512),
+    ([3, 700, 1, 0, 129], 200, 768),                  # K tail in the first GEMM
+])
+def test_ffn_dense_groups_elementwise(moe, sizes, d, F):
+    """R_max >= 1024 rows per expert selects the 2-CTA kernels."""
+    E = len(sizes)
+    R = sum(sizes)
+    offsets = np.array([0] + np.cumsum(sizes).tolist(), np.int32)
+    Xp = rand((R, d), 1.0, "bf16", 11)
+    W1 = rand((E, F, d), d ** -0.5, "bf16", 12)
+    W2 = rand((E, d, F), F ** -0.5, "bf16", 13)
+    Rmax = 1024 * E + 5
+    H, Yp = run_ffn(moe, Xp, W1, W2, offsets, Rmax)
+    Yr, Hr = oracle.expert_ffn(Xp, W1, W2, offsets, want_h=True)
+    assert_close(H[:R], Hr, "H")
+    assert_close(Yp[:R], Yr, "Yp")
     assert not H[R:].any() and not Yp[R:].any()
     assert moe.moe_device_error() == 0
 
