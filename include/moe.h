@@ -101,7 +101,10 @@ MOE_API int moe_gate(const void* x, const void* Wg, int dtype, int T, int d, int
  * section 2.1.2 (top-k gate); MoE-MPMC, problem statement (softmax router).
  *
  *   z[t][e] = logits[t][e] + bias[e]                (one fp32 addition)
- *   ids[t][0..k-1]  the k largest z, larger first; equal z: lower index first
+ *   ids[t][0..k-1]  the k largest z, larger first; equal z: lower index first.
+ *                   +0.0 and -0.0 are equal.  A NaN z ranks above every number
+ *                   (NaNs among themselves by index), so a diverged row still
+ *                   gets k distinct ids in [0, E); its weights are NaN.
  *   w[t][j]         = exp(z_j - z_0) / sum_{i<k} exp(z_i - z_0)  (fp32): the
  *                     k softmax probabilities renormalised to sum to 1
  *   counts[e]       tokens that chose e (demand, before drops)

@@ -14,7 +14,9 @@
 // U vectors per lane in flight, and
 //   dispatch: reads x[t] once and writes it to each of its kept rows;
 //   combine:  reads the token's kept rows of Yp, accumulates w_j * row in fp32
-//             with j ascending, and writes y[t] once.
+//             with j ascending, and writes y[t] once.  For k <= 8 the loads of
+//             all k rows of a column block are issued before the first
+//             multiply-add (one memory round trip per block instead of k).
 // Algorithmic bytes: dispatch T*d*s + R*d*s (+ T*k*4 index), combine
 // R*d*s + T*d*s (+ T*k*8 index/weights), s = element size.
 #include "common.cuh"
@@ -148,6 +150,87 @@ combine_kernel(const uint4* __restrict__ Yp, int T, int nvec, int k,
     }
 }
 
+// k <= KMAX: every kept row's CU vectors of a column block are in flight at
+// once; the sum is the same j-ascending fp32 sequence as combine_kernel's.
+template <int DT, int KMAX, int CU>
+__global__ void __launch_bounds__(kPermThreads)
+combine_wide_kernel(const uint4* __restrict__ Yp, int T, int nvec, int k,
+                    const int32_t* __restrict__ slot_row, const float* __restrict__ w,
+                    uint4* __restrict__ y, int R_max, int32_t* err) {
+    using V = Vec<DT>;
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int wpb = kPermThreads / 32;
+    const int nwarps = gridDim.x * wpb;
+    for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += nwarps) {
+        int my_row = -1;
+        float my_w = 0.0f;
+        if (lane < k) {
+            my_row = __ldg(slot_row + (size_t)t * k + lane);
+            my_w = w ? __ldg(w + (size_t)t * k + lane) : 1.0f;
+            if (my_row < -1 || my_row >= R_max) {
+                flag_error(err, MOE_DEVERR_ROW_INDEX);
+                my_row = -1;
+            }
+        }
+        int rows[KMAX];
+        float ws[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            rows[j] = __shfl_sync(0xffffffffu, my_row, j);  // lanes >= k hold -1
+            ws[j] = __shfl_sync(0xffffffffu, my_w, j);
+        }
+        uint4* dst = y + (size_t)t * nvec;
+        for (int c0 = 0; c0 < nvec; c0 += 32 * CU) {
+            uint4 v[KMAX][CU];
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+#pragma unroll
+                for (int u = 0; u < CU; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    v[j][u] = (rows[j] >= 0 && c < nvec)
+                                  ? ldg_nc_v4(Yp + (size_t)rows[j] * nvec + c)
+                                  : make_uint4(0, 0, 0, 0);
+                }
+            float acc[CU][V::N];
+#pragma unroll
+            for (int u = 0; u < CU; ++u)
+#pragma unroll
+                for (int i = 0; i < V::N; ++i) acc[u][i] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+                if (rows[j] >= 0) {
+#pragma unroll
+                    for (int u = 0; u < CU; ++u) V::fma(acc[u], ws[j], v[j][u]);
+                }
+#pragma unroll
+            for (int u = 0; u < CU; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < nvec) stg_v4(dst + c, V::pack(acc[u]));
+            }
+        }
+    }
+}
+
+// The combine (or dispatch-backward) launch for this k: the wide kernel up to
+// k = 8, the one-row-at-a-time kernel beyond.
+template <int DT>
+static int launch_combine(cudaStream_t st, int grid, const uint4* Yp, int T, int nvec, int k,
+                          const int32_t* slot_row, const float* w, uint4* y, int R_max) {
+    if (k <= 2)
+        return launch_pdl(combine_wide_kernel<DT, 2, 4>, grid, kPermThreads, 0, st, Yp, T, nvec,
+                          k, slot_row, w, y, R_max, device_error_word());
+    if (k <= 4)
+        return launch_pdl(combine_wide_kernel<DT, 4, 2>, grid, kPermThreads, 0, st, Yp, T, nvec,
+                          k, slot_row, w, y, R_max, device_error_word());
+    if (k <= 8)
+        return launch_pdl(combine_wide_kernel<DT, 8, 1>, grid, kPermThreads, 0, st, Yp, T, nvec,
+                          k, slot_row, w, y, R_max, device_error_word());
+    return launch_pdl(combine_kernel<DT>, grid, kPermThreads, 0, st, Yp, T, nvec, k, slot_row, w,
+                      y, R_max, device_error_word());
+}
+
 static int perm_grid(int T) {
     const int wpb = kPermThreads / 32;
     const int need = (T + wpb - 1) / wpb;
@@ -189,10 +272,13 @@ extern "C" MOE_API int moe_combine(const void* Yp, int dtype, int T, int d, int 
     if (T == 0) return MOE_OK;
     const int nvec = (int)((size_t)d * dtype_bytes(dtype) / 16);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    auto kern = dtype == MOE_DTYPE_BF16 ? combine_kernel<MOE_DTYPE_BF16>
-                                        : combine_kernel<MOE_DTYPE_F32>;
-    return launch_pdl(kern, perm_grid(T), kPermThreads, 0, st, static_cast<const uint4*>(Yp), T,
-                      nvec, k, slot_row, w, static_cast<uint4*>(y), R_max, device_error_word());
+    const uint4* src = static_cast<const uint4*>(Yp);
+    uint4* dst = static_cast<uint4*>(y);
+    if (dtype == MOE_DTYPE_BF16)
+        return launch_combine<MOE_DTYPE_BF16>(st, perm_grid(T), src, T, nvec, k, slot_row, w, dst,
+                                              R_max);
+    return launch_combine<MOE_DTYPE_F32>(st, perm_grid(T), src, T, nvec, k, slot_row, w, dst,
+                                         R_max);
 }
 
 extern "C" MOE_API int moe_dispatch_backward(const void* dXp, int dtype, int T, int d, int k,
@@ -204,9 +290,11 @@ extern "C" MOE_API int moe_dispatch_backward(const void* dXp, int dtype, int T, 
     if (T == 0) return MOE_OK;
     const int nvec = (int)((size_t)d * dtype_bytes(dtype) / 16);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    auto kern = dtype == MOE_DTYPE_BF16 ? combine_kernel<MOE_DTYPE_BF16>
-                                        : combine_kernel<MOE_DTYPE_F32>;
-    return launch_pdl(kern, perm_grid(T), kPermThreads, 0, st, static_cast<const uint4*>(dXp), T,
-                      nvec, k, slot_row, static_cast<const float*>(nullptr), static_cast<uint4*>(dx),
-                      R_max, device_error_word());
+    const uint4* src = static_cast<const uint4*>(dXp);
+    uint4* dst = static_cast<uint4*>(dx);
+    if (dtype == MOE_DTYPE_BF16)
+        return launch_combine<MOE_DTYPE_BF16>(st, perm_grid(T), src, T, nvec, k, slot_row,
+                                              nullptr, dst, R_max);
+    return launch_combine<MOE_DTYPE_F32>(st, perm_grid(T), src, T, nvec, k, slot_row, nullptr,
+                                         dst, R_max);
 }

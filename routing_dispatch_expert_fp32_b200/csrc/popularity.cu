@@ -8,8 +8,9 @@
 // experts ranked by window sum (desc), equal sums to the lower index.
 //
 // One CTA: thread e writes this step's count into ring row step % W, sums its
-// column over the n live rows (int64), writes the correctly rounded mean, and
-// ranks itself against every other expert's sum (E <= 1024, O(E^2 / threads)).
+// column over the n live rows (int64) and writes the correctly rounded mean;
+// then one warp per expert counts the experts ranked above it (32 sums per
+// lane pass, a warp sum), and the expert of rank r < P is hot[r].
 #include "common.cuh"
 
 namespace moe {
@@ -31,6 +32,7 @@ popularity_kernel(const int32_t* __restrict__ counts, int E, int32_t* __restrict
         const int32_t c = counts[e];
         hist[(size_t)slot * E + e] = c;
         long long sum = c;
+#pragma unroll 4
         for (long long i = 1; i < n; ++i) {
             const int s = (int)((step - i) % W);
             sum += hist[(size_t)s * E + e];
@@ -39,19 +41,29 @@ popularity_kernel(const int32_t* __restrict__ counts, int E, int32_t* __restrict
         mean[e] = __fdiv_rn(__ll2float_rn(sum), __ll2float_rn(n));
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    for (int e = threadIdx.x >> 5; e < E; e += nwarps) {
         const long long mine = s_sum[e];
-        int rank = 0;
-        for (int o = 0; o < E; ++o) {
+        int above = 0;
+        for (int o = lane; o < E; o += 32) {
             const long long v = s_sum[o];
-            rank += (v > mine) || (v == mine && o < e);
+            above += (v > mine) || (v == mine && o < e);
         }
-        if (rank < P) hot[rank] = e;
+        const int rank = __reduce_add_sync(0xffffffffu, above);
+        if (lane == 0 && rank < P) hot[rank] = e;
     }
     if (step_ptr) {
         __syncthreads();  // every thread has read the step
         if (threadIdx.x == 0) *step_ptr = step + 1;
     }
+}
+
+// A thread per expert for the window sums and a warp per expert (up to 32
+// warps) for the ranks.
+static int popularity_threads(int E) {
+    const int t = ((E + 31) / 32) * 32;
+    return t < 1024 ? (E < 32 ? 32 : (t * 4 < 1024 ? t * 4 : 1024)) : 1024;
 }
 
 }  // namespace moe
@@ -62,9 +74,9 @@ extern "C" MOE_API int moe_popularity_update(const int32_t* counts, int E, int32
     using namespace moe;
     if (E < 1 || E > kMaxExperts || W < 1 || step < 0 || P < 0 || P > E) return MOE_ERR_INVALID_ARG;
     if (!counts || !hist || !mean || (P > 0 && !hot)) return MOE_ERR_INVALID_ARG;
-    const int threads = ((E + 31) / 32) * 32;
-    return launch_pdl(popularity_kernel, 1, threads, 0, reinterpret_cast<cudaStream_t>(stream),
-                      counts, E, hist, W, (long long)step, (long long*)nullptr, mean, P, hot);
+    return launch_pdl(popularity_kernel, 1, popularity_threads(E), 0,
+                      reinterpret_cast<cudaStream_t>(stream), counts, E, hist, W, (long long)step,
+                      (long long*)nullptr, mean, P, hot);
 }
 
 extern "C" MOE_API int moe_popularity_update_dev(const int32_t* counts, int E, int32_t* hist, int W,
@@ -74,7 +86,7 @@ extern "C" MOE_API int moe_popularity_update_dev(const int32_t* counts, int E, i
     if (E < 1 || E > kMaxExperts || W < 1 || P < 0 || P > E) return MOE_ERR_INVALID_ARG;
     if (!counts || !hist || !mean || !step || (P > 0 && !hot)) return MOE_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(step) & 7u) != 0) return MOE_ERR_UNSUPPORTED;
-    const int threads = ((E + 31) / 32) * 32;
-    return launch_pdl(popularity_kernel, 1, threads, 0, reinterpret_cast<cudaStream_t>(stream),
-                      counts, E, hist, W, 0LL, reinterpret_cast<long long*>(step), mean, P, hot);
+    return launch_pdl(popularity_kernel, 1, popularity_threads(E), 0,
+                      reinterpret_cast<cudaStream_t>(stream), counts, E, hist, W, 0LL,
+                      reinterpret_cast<long long*>(step), mean, P, hot);
 }

@@ -3,22 +3,31 @@
 // "A Survey on Mixture of Experts", section 5 (gate routing; tokens dispatched
 // under an expert-capacity limit) and PopFetcher, section 2.1.2 (top-k gate).
 //
-// Three launches, no inter-CTA waiting:
-//   K1 route_topk    one CTA of 32 warps (8 for E > 256) per chunk of 256 tokens (8 per warp;
-//                    the next token's logits are loaded while the current one
-//                    is ranked).  A group of L lanes
-//                    (L = 8, 16 or 32) scores one token: each lane holds E/L
-//                    of the fp32 keys z = logit + bias (coalesced loads), k
-//                    rounds of a butterfly argmax under the total order
-//                    (z desc, index asc) pick the experts, lane j keeps slot j
-//                    and computes w_j = exp(z_j - z_0) / sum_i exp(z_i - z_0).
-//                    Per-chunk expert histogram in shared memory (atomicAdd
-//                    on counts commutes, so the result is order-free).
-//   K2 route_scan    one CTA: per expert, exclusive prefix of the chunk
-//                    histograms (two-level: segments of chunks, then chunks),
-//                    counts, kept = min(counts, capacity), offsets = exclusive
-//                    scan of kept, n_dropped.
-//   K3 route_assign  one CTA per chunk again (a token per thread); a slot's position inside its
+// Ranking: z = logit + bias (one fp32 add) is mapped to a 32-bit key whose
+// unsigned order is the order (z desc): -0.0 is folded onto +0.0 (they tie),
+// and every NaN gets the largest key (a NaN ranks above every number, as in
+// torch.topk), so each of the k rounds picks an expert in [0, E) whatever the
+// input.  Equal keys go to the lower expert index.
+//
+// Three launches, no inter-CTA waiting (chunks of 256 tokens):
+//   K1 route_topk    one CTA per chunk.  E <= 32: one token per thread; the
+//                    row's keys sit in registers (16-byte loads when E % 4 == 0)
+//                    and k passes of an unrolled max pick the experts.  E > 32:
+//                    one token per warp, lane l holding experts
+//                    (i / V) * 32V + l * V + i % V (V-wide vector loads), with
+//                    the next tokens' logits loaded while the current one is
+//                    ranked; per round the largest key by a warp reduction, then
+//                    the lowest index among the lanes holding it.  Weights
+//                    w_j = exp(z_j - z_0) / sum_i exp(z_i - z_0), the sum in rank
+//                    order.  Per-chunk expert histogram in shared memory
+//                    (atomicAdd on counts commutes: the result is order-free).
+//   K2 route_scan    one CTA per 32 experts: per expert, the exclusive prefix of
+//                    the chunk histograms over chunks (32 warps each sum a
+//                    segment of chunks, then the segments are scanned), counts,
+//                    kept = min(counts, capacity).
+//   K3 route_assign  one CTA per chunk (a token per thread); offsets = exclusive
+//                    scan of kept (every CTA scans the E values itself; CTA 0
+//                    writes offsets and n_dropped); a slot's position inside its
 //                    expert = chunk base + slots of earlier warps of the chunk
 //                    + earlier lanes of its warp, all from per-warp lane masks
 //                    (atomicOr commutes; popc of the lower-lane bits gives the
@@ -30,21 +39,19 @@
 namespace moe {
 
 constexpr int kChunk = 256;        // tokens per chunk (= per CTA in K1 and K3)
-// K1 threads: 32 warps (kChunk / 32 tokens each); 8 warps when a lane holds
-// 16 or more keys, so the keys of two tokens stay in registers.
-template <int VPL>
-constexpr int topk_threads() { return VPL >= 16 ? 256 : 1024; }
-constexpr int kThreads = kChunk;   // K3: one token per thread
+constexpr int kThreads = kChunk;   // K3 (and K1 for E <= 32): one token per thread
 constexpr int kWarps = kThreads / 32;
 constexpr int kScanThreads = 1024;
 
-__device__ __forceinline__ bool key_better(float av, int ai, float bv, int bi) {
-    return av > bv || (av == bv && ai < bi);
-}
+// K1 threads for E > 32: 32 warps of 8 tokens; 8 warps of 32 tokens when a
+// lane holds 16 or more keys (register budget).
+template <int VPL>
+constexpr int warp_topk_threads() { return VPL >= 16 ? 256 : 1024; }
 
-// Order-preserving map of a finite fp32 to uint32 (larger float -> larger
-// key); -0.0 is folded onto +0.0 first so that the two still tie.
-__device__ __forceinline__ uint32_t order_key(float z) {
+// Order key of z: larger z -> larger key; -0.0 ties with +0.0; NaN above all.
+// Keys of numbers are >= 0x007FFFFF (that of -inf), so 0 is free as "none".
+__device__ __forceinline__ uint32_t route_key(float z) {
+    if (z != z) return 0xFFFFFFFFu;
     const uint32_t u = __float_as_uint(z == 0.0f ? 0.0f : z);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
@@ -53,248 +60,333 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 }
 
 // ------------------------------------------------------------------- K1 ----
-template <int L, int VPL>
-__global__ void __launch_bounds__(topk_threads<VPL>())
-route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
-                  int k, int32_t* __restrict__ ids, float* __restrict__ w,
-                  int32_t* __restrict__ chunk_hist) {
-    __shared__ int s_hist[kMaxExperts];
-    constexpr int kTopkThreads = topk_threads<VPL>();
-    for (int e = threadIdx.x; e < E; e += kTopkThreads) s_hist[e] = 0;
-    __syncthreads();
+// E <= EMAX <= 32: one token per thread.  KMAX >= k bounds the unrolled
+// rounds; vw (1, 2 or 4) is the load width (the host checks E % vw == 0 and the
+// alignment of `logits`).
+template <int EMAX, int KMAX>
+__global__ void __launch_bounds__(kThreads)
+route_topk_lane_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
+                       int E, int k, int vw, int32_t* __restrict__ ids, float* __restrict__ w,
+                       int32_t* __restrict__ chunk_hist, int32_t* err) {
+    __shared__ int s_hist[EMAX];
+    __shared__ float s_bias[EMAX];
     pdl_wait();
     pdl_trigger();
+    if (threadIdx.x < EMAX) {
+        s_hist[threadIdx.x] = 0;
+        s_bias[threadIdx.x] =
+            (bias != nullptr && (int)threadIdx.x < E) ? bias[threadIdx.x] : 0.0f;
+    }
+    __syncthreads();
+    const int t = blockIdx.x * kChunk + threadIdx.x;
+    if (t < T) {
+        const float* row = logits + (size_t)t * E;
+        float z[EMAX];
+        if (vw == 4) {
+#pragma unroll
+            for (int q = 0; q < EMAX / 4; ++q) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (4 * q < E) v = __ldg(reinterpret_cast<const float4*>(row) + q);
+                z[4 * q] = v.x; z[4 * q + 1] = v.y; z[4 * q + 2] = v.z; z[4 * q + 3] = v.w;
+            }
+        } else if (vw == 2) {
+#pragma unroll
+            for (int q = 0; q < EMAX / 2; ++q) {
+                float2 v = make_float2(0.f, 0.f);
+                if (2 * q < E) v = __ldg(reinterpret_cast<const float2*>(row) + q);
+                z[2 * q] = v.x; z[2 * q + 1] = v.y;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e) z[e] = (e < E) ? __ldg(row + e) : 0.0f;
+        }
+        uint32_t key[EMAX];
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) key[e] = (e < E) ? route_key(__fadd_rn(z[e], s_bias[e])) : 0u;
 
-    constexpr int G = 32 / L;                          // tokens per warp per iteration
-    constexpr int kPerWarp = kChunk / (kTopkThreads / 32);
-    constexpr int kIters = kPerWarp / G;
+        int si[KMAX];
+        float ex[KMAX];
+        float z0 = 0.0f, s = 0.0f;
+#pragma unroll
+        for (int r = 0; r < KMAX; ++r) {
+            si[r] = 0;
+            ex[r] = 0.0f;
+            if (r < k) {
+                // strict '>' scanning upward: equal keys keep the lower index
+                uint32_t bk = 0u;
+                int bi = 0;
+#pragma unroll
+                for (int e = 0; e < EMAX; ++e)
+                    if (key[e] > bk) {
+                        bk = key[e];
+                        bi = e;
+                    }
+#pragma unroll
+                for (int e = 0; e < EMAX; ++e)
+                    if (e == bi) key[e] = 0u;
+                const float zr = key_value(bk);
+                if (r == 0) z0 = zr;
+                si[r] = bi;
+                ex[r] = expf(__fsub_rn(zr, z0));
+                s = __fadd_rn(s, ex[r]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < KMAX; ++r) {
+            if (r < k) {
+                ids[(size_t)t * k + r] = si[r];
+                w[(size_t)t * k + r] = __fdiv_rn(ex[r], s);
+                if (si[r] < E) atomicAdd(&s_hist[si[r]], 1);
+                else flag_error(err, MOE_DEVERR_EXPERT_INDEX);
+            }
+        }
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < E) chunk_hist[(size_t)blockIdx.x * E + threadIdx.x] = s_hist[threadIdx.x];
+}
+
+// E > 32: one token per warp; each lane holds VPL keys, loaded VW floats at a
+// time: slot i of lane l is expert (i / VW) * 32 * VW + l * VW + i % VW, which
+// grows with i, so a lane's strict '>' scan keeps the lowest index of a tie.
+template <int VPL, int VW>
+__device__ __forceinline__ void load_lane(const float* __restrict__ row, int lane_vw, int E,
+                                          float (&v)[VPL]) {
+#pragma unroll
+    for (int g = 0; g < VPL / VW; ++g) {
+        const int e = g * 32 * VW + lane_vw;
+        if constexpr (VW == 4) {
+            float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (e < E) q = __ldg(reinterpret_cast<const float4*>(row + e));
+            v[4 * g] = q.x; v[4 * g + 1] = q.y; v[4 * g + 2] = q.z; v[4 * g + 3] = q.w;
+        } else if constexpr (VW == 2) {
+            float2 q = make_float2(0.f, 0.f);
+            if (e < E) q = __ldg(reinterpret_cast<const float2*>(row + e));
+            v[2 * g] = q.x; v[2 * g + 1] = q.y;
+        } else {
+            v[g] = (e < E) ? __ldg(row + e) : 0.0f;
+        }
+    }
+}
+
+template <int VPL, int VW>
+__global__ void __launch_bounds__(warp_topk_threads<VPL>())
+route_topk_warp_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
+                       int E, int k, int32_t* __restrict__ ids, float* __restrict__ w,
+                       int32_t* __restrict__ chunk_hist, int32_t* err) {
+    constexpr int kT = warp_topk_threads<VPL>();
+    constexpr int kPerWarp = kChunk / (kT / 32);           // tokens per warp
+    constexpr int D = VPL <= 4 ? 2 : 1;                    // tokens in flight per warp
+    static_assert(kPerWarp % D == 0, "token groups");
+    __shared__ int s_hist[kMaxExperts];
+    pdl_wait();
+    pdl_trigger();
+    for (int e = threadIdx.x; e < E; e += kT) s_hist[e] = 0;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane / L, gl = lane % L;
-
-    // this lane's experts are gl, gl + L, gl + 2L, ...
+    const int lane_vw = lane * VW;
     float b[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-        const int e = gl + i * L;
-        b[i] = (bias != nullptr && e < E) ? bias[e] : 0.0f;
+        const int e = (i / VW) * 32 * VW + lane_vw + i % VW;
+        b[i] = (bias != nullptr && e < E) ? __ldg(bias + e) : 0.0f;
     }
+    __syncthreads();
 
     const int t_warp = blockIdx.x * kChunk + warp * kPerWarp;
-    float zn[VPL];  // logits of the next token of this group, in flight
-    {
-        const int t = min(t_warp + g, T - 1);
+    float cur[D][VPL], nxt[D][VPL];
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const int e = gl + i * L;
-            zn[i] = (e < E) ? __ldg(logits + (size_t)t * E + e) : 0.0f;
-        }
+    for (int u = 0; u < D; ++u) {
+        const int t = t_warp + u;
+        if (t < T) load_lane<VPL, VW>(logits + (size_t)t * E, lane_vw, E, cur[u]);
     }
 #pragma unroll 1
-    for (int it = 0; it < kIters; ++it) {
-        const int t = t_warp + it * G + g;
-        const bool active = t < T;
-        float z[VPL];
+    for (int g = 0; g < kPerWarp / D; ++g) {
+        if (g + 1 < kPerWarp / D) {
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const int e = gl + i * L;
-            z[i] = (e < E) ? __fadd_rn(zn[i], b[i]) : -INFINITY;
-        }
-        if (it + 1 < kIters) {
-            const int tn = min(t + G, T - 1);
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int e = gl + i * L;
-                zn[i] = (e < E) ? __ldg(logits + (size_t)tn * E + e) : 0.0f;
+            for (int u = 0; u < D; ++u) {
+                const int t = t_warp + (g + 1) * D + u;
+                if (t < T) load_lane<VPL, VW>(logits + (size_t)t * E, lane_vw, E, nxt[u]);
             }
         }
-
-        uint32_t taken = 0;
-        float my_z = 0.0f;
-        int my_e = 0;
-        if constexpr (L == 32) {
-            // One token per warp: per round, the largest order key by a warp
-            // reduction, then the lowest expert index among the lanes holding
-            // it (each lane's candidate is its own lowest-index maximum).
-            uint32_t key[VPL];
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) key[i] = (gl + i * L < E) ? order_key(z[i]) : 0u;
-            for (int r = 0; r < k; ++r) {
-                uint32_t bk = 0u;
-                int bi = INT_MAX;
+        for (int u = 0; u < D; ++u) {
+            const int t = t_warp + g * D + u;
+            if (t < T) {  // warp-uniform
+                uint32_t key[VPL];
 #pragma unroll
                 for (int i = 0; i < VPL; ++i) {
-                    if (!((taken >> i) & 1u) && key[i] > bk) {
-                        bk = key[i];
-                        bi = gl + i * L;
-                    }
+                    const int e = (i / VW) * 32 * VW + lane_vw + i % VW;
+                    key[i] = (e < E) ? route_key(__fadd_rn(cur[u][i], b[i])) : 0u;
                 }
-                const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
-                const int win = (int)__reduce_min_sync(0xffffffffu, bk == m ? (uint32_t)bi : 0xffffffffu);
-                if (win % L == gl) taken |= 1u << (win / L);
-                if (gl == r) {
-                    my_z = key_value(m);
-                    my_e = win;
-                }
-            }
-        } else {
-            for (int r = 0; r < k; ++r) {
-                float bv = -INFINITY;
-                int bi = INT_MAX;
+                float my_z = 0.0f;
+                int my_e = 0;
+                for (int r = 0; r < k; ++r) {
+                    uint32_t bk = 0u;
+                    int bi = INT_MAX;
 #pragma unroll
-                for (int i = 0; i < VPL; ++i) {
-                    const int e = gl + i * L;
-                    if (e < E && !((taken >> i) & 1u) && key_better(z[i], e, bv, bi)) {
-                        bv = z[i];
-                        bi = e;
-                    }
-                }
+                    for (int i = 0; i < VPL; ++i)
+                        if (key[i] > bk) {
+                            bk = key[i];
+                            bi = (i / VW) * 32 * VW + lane_vw + i % VW;
+                        }
+                    // k <= E, so some lane still holds an untaken expert: m > 0
+                    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+                    const int win = (int)__reduce_min_sync(
+                        0xffffffffu, bk == m ? (uint32_t)bi : 0xffffffffu);
+                    const int off = win - lane_vw;  // slot of the winner in its lane
 #pragma unroll
-                for (int off = L / 2; off > 0; off >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off, L);
-                    const int oi = __shfl_xor_sync(0xffffffffu, bi, off, L);
-                    if (key_better(ov, oi, bv, bi)) {
-                        bv = ov;
-                        bi = oi;
+                    for (int i = 0; i < VPL; ++i)
+                        if (off == (i / VW) * 32 * VW + i % VW) key[i] = 0u;
+                    if (lane == r) {
+                        my_z = key_value(m);
+                        my_e = win;
                     }
                 }
-                // every lane of the group now holds the same winner
-                if (bi % L == gl) taken |= 1u << (bi / L);
-                if (gl == r) {
-                    my_z = bv;
-                    my_e = bi;
+                const float z0 = __shfl_sync(0xffffffffu, my_z, 0);
+                const float ex = (lane < k) ? expf(__fsub_rn(my_z, z0)) : 0.0f;
+                float s = 0.0f;
+                for (int i = 0; i < k; ++i) s = __fadd_rn(s, __shfl_sync(0xffffffffu, ex, i));
+                if (lane < k) {
+                    ids[(size_t)t * k + lane] = my_e;
+                    w[(size_t)t * k + lane] = __fdiv_rn(ex, s);
+                    if ((unsigned)my_e < (unsigned)E) atomicAdd(&s_hist[my_e], 1);
+                    else flag_error(err, MOE_DEVERR_EXPERT_INDEX);
                 }
             }
         }
-
-        const float z0 = __shfl_sync(0xffffffffu, my_z, 0, L);
-        const float ex = (gl < k) ? expf(__fsub_rn(my_z, z0)) : 0.0f;
-        float s = 0.0f;
-        for (int i = 0; i < k; ++i) s = __fadd_rn(s, __shfl_sync(0xffffffffu, ex, i, L));
-        if (active && gl < k) {
-            ids[(size_t)t * k + gl] = my_e;
-            w[(size_t)t * k + gl] = __fdiv_rn(ex, s);
-            atomicAdd(&s_hist[my_e], 1);
+        if (g + 1 < kPerWarp / D) {
+#pragma unroll
+            for (int u = 0; u < D; ++u)
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) cur[u][i] = nxt[u][i];
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += kTopkThreads)
+    for (int e = threadIdx.x; e < E; e += kT)
         chunk_hist[(size_t)blockIdx.x * E + e] = s_hist[e];
 }
 
 // ------------------------------------------------------------------- K2 ----
+// One CTA per 32 experts (lane = expert); warp s sums chunks
+// [s * cps, (s + 1) * cps), the 32 segment totals are scanned per expert, and
+// each warp rescans its segment to write the chunk bases.
 __global__ void __launch_bounds__(kScanThreads)
-route_scan_kernel(const int32_t* __restrict__ chunk_hist, int nchunks, int T, int E, int k,
-                  int capacity, int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
-                  int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
-                  int32_t* __restrict__ n_dropped) {
-    __shared__ int32_t s_seg[kScanThreads];  // [segment][expert]
-    __shared__ int32_t s_warp[kScanThreads / 32];
+route_scan_kernel(const int32_t* __restrict__ chunk_hist, int nchunks, int E, int capacity,
+                  int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
+                  int32_t* __restrict__ kept) {
+    __shared__ int32_t s_seg[32][33];
     pdl_wait();
     pdl_trigger();
-    const int tid = threadIdx.x;
-    const int S = kScanThreads / E;              // segments (E <= 1024 so S >= 1)
-    const int cps = (nchunks + S - 1) / S;       // chunks per segment
-    const int e = tid % E, seg = tid / E;
-    const bool worker = seg < S;
-    const int c0 = seg * cps, c1 = min(nchunks, c0 + cps);
-
-    // phase 1: per (segment, expert) totals
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int e = blockIdx.x * 32 + lane;
+    const bool ok = e < E;
+    const int cps = (nchunks + 31) / 32;
+    const int c0 = wid * cps, c1 = min(nchunks, c0 + cps);
     int32_t part = 0;
-    if (worker) {
-#pragma unroll 8
+    if (ok) {
+#pragma unroll 4
         for (int c = c0; c < c1; ++c) part += chunk_hist[(size_t)c * E + e];
     }
-    if (worker) s_seg[seg * E + e] = part;
+    s_seg[wid][lane] = part;
     __syncthreads();
-
-    // phase 2: per expert, exclusive over segments; totals are the counts
-    int32_t my_kept = 0;
-    if (tid < E) {
+    if (wid == 0) {
         int32_t run = 0;
-        for (int s = 0; s < S; ++s) {
-            const int32_t v = s_seg[s * E + tid];
-            s_seg[s * E + tid] = run;
+        for (int s = 0; s < 32; ++s) {
+            const int32_t v = s_seg[s][lane];
+            s_seg[s][lane] = run;
             run += v;
         }
-        counts[tid] = run;
-        my_kept = (capacity > 0 && run > capacity) ? capacity : run;
-        kept[tid] = my_kept;
+        if (ok) {
+            counts[e] = run;
+            kept[e] = (capacity > 0 && run > capacity) ? capacity : run;
+        }
     }
     __syncthreads();
-
-    // phase 3: per chunk bases
-    if (worker) {
-        int32_t run = s_seg[seg * E + e];
-#pragma unroll 8
+    if (ok) {
+        int32_t run = s_seg[wid][lane];
+#pragma unroll 4
         for (int c = c0; c < c1; ++c) {
             const int32_t v = chunk_hist[(size_t)c * E + e];
             chunk_base[(size_t)c * E + e] = run;
             run += v;
         }
     }
-
-    // exclusive scan of kept over experts (block scan; tid >= E contributes 0)
-    const int lane = tid & 31, wid = tid >> 5;
-    int32_t incl = my_kept;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-    }
-    if (lane == 31) s_warp[wid] = incl;
-    __syncthreads();
-    if (wid == 0) {
-        int32_t v = s_warp[lane];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int32_t o = __shfl_up_sync(0xffffffffu, v, off);
-            if (lane >= off) v += o;
-        }
-        s_warp[lane] = v;  // inclusive over warps
-    }
-    __syncthreads();
-    const int32_t before = (wid > 0 ? s_warp[wid - 1] : 0) + incl - my_kept;
-    if (tid < E) offsets[tid] = before;
-    if (tid == 0) {
-        const int32_t total = s_warp[31];
-        offsets[E] = total;
-        n_dropped[0] = (int32_t)((int64_t)T * k - total);
-    }
 }
 
 // ------------------------------------------------------------------- K3 ----
 __global__ void __launch_bounds__(kThreads)
 route_assign_kernel(const int32_t* __restrict__ ids, int T, int E, int k, int capacity,
-                    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
-                    int32_t* __restrict__ slot_row, int32_t* __restrict__ row_slot) {
+                    int nchunks, const int32_t* __restrict__ chunk_base,
+                    const int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
+                    int32_t* __restrict__ n_dropped, int32_t* __restrict__ slot_row,
+                    int32_t* __restrict__ row_slot, int32_t* err) {
     __shared__ uint32_t s_mask[kWarps][kMaxExperts];
     __shared__ int32_t s_base[kMaxExperts];
-    __shared__ int32_t s_off[kMaxExperts];
+    __shared__ int32_t s_off[kMaxExperts + 1];
+    __shared__ int32_t s_warp[kWarps];
     pdl_wait();
     pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // offsets: exclusive scan of kept over the experts, per = experts a thread holds
+    const int per = (E + kThreads - 1) / kThreads;
+    const int e0 = tid * per;
+    int32_t loc = 0;
+    for (int i = 0; i < per; ++i)
+        if (e0 + i < E) loc += kept[e0 + i];
+    int32_t incl = loc;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_warp[warp] = incl;
     for (int e = tid; e < E; e += kThreads) {
-        s_base[e] = chunk_base[(size_t)blockIdx.x * E + e];
-        s_off[e] = offsets[e];
+        s_base[e] = blockIdx.x < nchunks ? chunk_base[(size_t)blockIdx.x * E + e] : 0;
 #pragma unroll
         for (int wv = 0; wv < kWarps; ++wv) s_mask[wv][e] = 0u;
     }
     __syncthreads();
+    int32_t run = incl - loc;
+    int32_t total = 0;
+#pragma unroll
+    for (int wv = 0; wv < kWarps; ++wv) {
+        if (wv < warp) run += s_warp[wv];
+        total += s_warp[wv];
+    }
+    for (int i = 0; i < per; ++i)
+        if (e0 + i < E) {
+            s_off[e0 + i] = run;
+            run += kept[e0 + i];
+        }
+    if (tid == 0) s_off[E] = total;
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        for (int e = tid; e <= E; e += kThreads) offsets[e] = s_off[e];
+        if (tid == 0) n_dropped[0] = (int32_t)((int64_t)T * k - total);
+    }
 
-    const int t = blockIdx.x * kChunk + warp * 32 + lane;
+    const int t = blockIdx.x * kChunk + tid;
     const bool active = t < T;
     const int32_t* my_ids = ids + (size_t)t * k;
     if (active)
-        for (int j = 0; j < k; ++j) atomicOr(&s_mask[warp][my_ids[j]], 1u << lane);
+        for (int j = 0; j < k; ++j) {
+            const int e = my_ids[j];
+            if ((unsigned)e < (unsigned)E) atomicOr(&s_mask[warp][e], 1u << lane);
+        }
     __syncthreads();
 
     if (active) {
         const uint32_t lower = (1u << lane) - 1u;
         for (int j = 0; j < k; ++j) {
             const int e = my_ids[j];
+            const int32_t s = t * k + j;
+            if ((unsigned)e >= (unsigned)E) {
+                flag_error(err, MOE_DEVERR_EXPERT_INDEX);
+                slot_row[s] = -1;
+                continue;
+            }
             int32_t p = s_base[e] + __popc(s_mask[warp][e] & lower);
             for (int wv = 0; wv < warp; ++wv) p += __popc(s_mask[wv][e]);
-            const int32_t s = t * k + j;
             if (capacity <= 0 || p < capacity) {
                 const int32_t r = s_off[e] + p;
                 slot_row[s] = r;
@@ -308,11 +400,28 @@ route_assign_kernel(const int32_t* __restrict__ ids, int T, int E, int k, int ca
 
 static size_t align256(size_t v) { return (v + 255u) & ~size_t(255u); }
 
-template <int L, int VPL>
-static int launch_topk(int nchunks, cudaStream_t st, const float* logits, const float* bias,
-                       int T, int E, int k, int32_t* ids, float* w, int32_t* hist) {
-    return launch_pdl(route_topk_kernel<L, VPL>, nchunks, topk_threads<VPL>(), 0, st, logits, bias,
-                      T, E, k, ids, w, hist);
+template <int EMAX, int KMAX>
+static int launch_lane(int nchunks, cudaStream_t st, const float* logits, const float* bias,
+                       int T, int E, int k, int vw, int32_t* ids, float* w, int32_t* hist) {
+    return launch_pdl(route_topk_lane_kernel<EMAX, KMAX>, nchunks, kThreads, 0, st, logits, bias,
+                      T, E, k, vw, ids, w, hist, device_error_word());
+}
+template <int EMAX>
+static int launch_lane_k(int nchunks, cudaStream_t st, const float* logits, const float* bias,
+                         int T, int E, int k, int vw, int32_t* ids, float* w, int32_t* hist) {
+    if (k <= 2) return launch_lane<EMAX, 2>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
+    if (k <= 8) return launch_lane<EMAX, 8>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
+    return launch_lane<EMAX, EMAX>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
+}
+template <int VPL>
+static int launch_warp(int nchunks, cudaStream_t st, const float* logits, const float* bias,
+                       int T, int E, int k, bool vec, int32_t* ids, float* w, int32_t* hist) {
+    constexpr int VW = VPL >= 4 ? 4 : VPL;
+    if (vec)
+        return launch_pdl(route_topk_warp_kernel<VPL, VW>, nchunks, warp_topk_threads<VPL>(), 0,
+                          st, logits, bias, T, E, k, ids, w, hist, device_error_word());
+    return launch_pdl(route_topk_warp_kernel<VPL, 1>, nchunks, warp_topk_threads<VPL>(), 0, st,
+                      logits, bias, T, E, k, ids, w, hist, device_error_word());
 }
 
 // The three launches of one routing call; `scratch` is 256-byte aligned and
@@ -330,26 +439,29 @@ static int launch_route(const float* logits, const float* bias, int T, int E, in
     int32_t* hist = reinterpret_cast<int32_t*>(scratch);
     int32_t* base = reinterpret_cast<int32_t*>(scratch + align256((size_t)nchunks * E * 4));
     if (T > 0) {
+        // widest load the row layout and the pointer's alignment allow
+        const uintptr_t p = reinterpret_cast<uintptr_t>(logits);
+        const int vw = (E % 4 == 0 && p % 16 == 0) ? 4 : (E % 2 == 0 && p % 8 == 0) ? 2 : 1;
         int rc;
-        if (E <= 8) rc = launch_topk<8, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 16) rc = launch_topk<16, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 32) rc = launch_topk<32, 1>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 64) rc = launch_topk<32, 2>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 128) rc = launch_topk<32, 4>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 256) rc = launch_topk<32, 8>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else if (E <= 512) rc = launch_topk<32, 16>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
-        else rc = launch_topk<32, 32>(nchunks, st, logits, bias, T, E, k, ids, w, hist);
+        if (E <= 8) rc = launch_lane_k<8>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
+        else if (E <= 16) rc = launch_lane_k<16>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
+        else if (E <= 32) rc = launch_lane_k<32>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
+        else if (E <= 64) rc = launch_warp<2>(nchunks, st, logits, bias, T, E, k, vw >= 2, ids, w, hist);
+        else if (E <= 128) rc = launch_warp<4>(nchunks, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
+        else if (E <= 256) rc = launch_warp<8>(nchunks, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
+        else if (E <= 512) rc = launch_warp<16>(nchunks, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
+        else rc = launch_warp<32>(nchunks, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
         if (rc != MOE_OK) return MOE_ERR_CUDA;
     }
-    if (launch_pdl(route_scan_kernel, 1, kScanThreads, 0, st, (const int32_t*)hist, nchunks, T, E,
-                   k, capacity, base, counts, kept, offsets, n_dropped) != MOE_OK)
+    if (launch_pdl(route_scan_kernel, (E + 31) / 32, kScanThreads, 0, st, (const int32_t*)hist,
+                   nchunks, E, capacity, base, counts, kept) != MOE_OK)
         return MOE_ERR_CUDA;
-    if (T > 0) {
-        if (launch_pdl(route_assign_kernel, nchunks, kThreads, 0, st, (const int32_t*)ids, T, E, k,
-                       capacity, (const int32_t*)base, (const int32_t*)offsets, slot_row,
-                       row_slot) != MOE_OK)
-            return MOE_ERR_CUDA;
-    }
+    // at least one CTA: it writes offsets and n_dropped even when T = 0
+    if (launch_pdl(route_assign_kernel, nchunks > 0 ? nchunks : 1, kThreads, 0, st,
+                   (const int32_t*)ids, T, E, k, capacity, nchunks, (const int32_t*)base,
+                   (const int32_t*)kept, offsets, n_dropped, slot_row, row_slot,
+                   device_error_word()) != MOE_OK)
+        return MOE_ERR_CUDA;
     return MOE_OK;
 }
 
@@ -412,17 +524,18 @@ namespace moe {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB on every device
 static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
 
+// Device address of the array on the current device, looked up once per device
+// (host threads that race on the first lookup store the same address).
 static void* noalloc_scratch_ptr() {
-    constexpr int kMaxDevices = 64;
-    static void* cache[kMaxDevices] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!cache[dev]) {
-        void* p = nullptr;
+    static std::atomic<void*> cache[kMaxDevices] = {};
+    const int dev = current_device();
+    if (dev < 0) return nullptr;
+    void* p = cache[dev].load(std::memory_order_acquire);
+    if (!p) {
         if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
-        cache[dev] = p;
+        cache[dev].store(p, std::memory_order_release);
     }
-    return cache[dev];
+    return p;
 }
 
 }  // namespace moe

@@ -116,3 +116,67 @@ def test_route_is_deterministic(moe):
     for other in runs[1:]:
         for name in runs[0]:
             assert np.array_equal(runs[0][name], other[name]), name
+
+
+def _with_nans(rng, T, E, frac):
+    """Logits N(0,1) with a fraction of entries replaced by NaNs of several bit
+    patterns (quiet, negative, all-ones) and infinities; some rows all NaN and
+    some with fewer than k numbers."""
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    bits = np.array([0x7FC00000, 0xFFC00000, 0xFFFFFFFF, 0x7F800001], np.uint32).view(np.float32)
+    special = np.concatenate([bits, np.array([np.inf, -np.inf], np.float32)])
+    mask = rng.random((T, E)) < frac
+    lg[mask] = special[rng.integers(0, len(special), int(mask.sum()))]
+    lg[0] = np.nan
+    lg[1, 1:] = np.nan
+    lg[2, : E - 1] = -np.inf
+    return lg
+
+
+@pytest.mark.parametrize("T,E,k,cap", [(600, 8, 2, 0), (600, 16, 3, 90), (513, 24, 4, 0),
+                                       (777, 64, 2, 30), (1100, 128, 4, 0), (300, 256, 8, 0)])
+def test_route_nan_logits_rank_first_and_stay_in_range(moe, T, E, k, cap):
+    """NaN scores rank above every number, NaNs among themselves by index (the
+    oracle's reading); every id stays in [0, E) and routing is bit-exact."""
+    rng = np.random.default_rng(T + E)
+    logits = _with_nans(rng, T, E, 0.1)
+    g = run_route(moe, logits, None, k, cap)
+    r = oracle.route(logits, None, k, cap)
+    R = int(r["offsets"][-1])
+    for name in ["ids", "counts", "kept", "offsets", "slot_row"]:
+        assert np.array_equal(g[name], r[name]), name
+    assert np.array_equal(g["row_slot"][:R], r["row_slot"])
+    assert int(g["n_dropped"][0]) == r["n_dropped"]
+    assert g["ids"].min() >= 0 and g["ids"].max() < E
+    np.testing.assert_allclose(g["w"], r["w"], rtol=4e-6, atol=1e-8, equal_nan=True)
+    assert np.array_equal(np.isnan(g["w"]), np.isnan(r["w"]))
+    assert moe.moe_device_error() == 0
+
+
+@pytest.mark.parametrize("E", [8, 20, 40, 128])
+def test_route_unaligned_logits_take_the_scalar_loads(moe, E):
+    """A logits pointer that is not 16-byte aligned (an offset view) routes the
+    same as an aligned copy."""
+    rng = np.random.default_rng(E)
+    T, k = 300, 2
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    flat = torch.empty(T * E + 1, device="cuda")
+    view = flat[1:].view(T, E)
+    view.copy_(dev(logits))
+    i32 = torch.int32
+    out = dict(ids=torch.empty((T, k), dtype=i32, device="cuda"),
+               w=torch.empty((T, k), device="cuda"),
+               counts=torch.empty((E,), dtype=i32, device="cuda"),
+               kept=torch.empty((E,), dtype=i32, device="cuda"),
+               offsets=torch.empty((E + 1,), dtype=i32, device="cuda"),
+               slot_row=torch.empty((T, k), dtype=i32, device="cuda"),
+               row_slot=torch.empty((T * k,), dtype=i32, device="cuda"),
+               n_dropped=torch.empty((1,), dtype=i32, device="cuda"))
+    ws = torch.empty(moe.moe_route_workspace_size(T, E, k), dtype=torch.uint8, device="cuda")
+    moe.moe_route(view, None, k, 0, out["ids"], out["w"], out["counts"], out["kept"],
+                  out["offsets"], out["slot_row"], out["row_slot"], out["n_dropped"], ws)
+    torch.cuda.synchronize()
+    r = oracle.route(logits, None, k, 0)
+    for name in ["ids", "counts", "offsets", "slot_row"]:
+        assert np.array_equal(host(out[name]), r[name]), name
+    np.testing.assert_allclose(host(out["w"]), r["w"], rtol=4e-6, atol=1e-8)
