@@ -13,6 +13,12 @@ per-rank batches: weak scaling) the time is the max over ranks and the only
 collective in a step is the all_reduce of the per-expert counts that keeps the
 popularity statistic global.
 
+The headline line is the largest single-GPU workload (fine_grained: T=32768,
+d=4096, E=256, k=8, F=1024).  With one rank the line also carries, under
+extras.workloads, the same measurement of multistep_window (all 8 steps, the
+popularity window and top-8 on) and of the bandwidth sweep at T=65536 with and
+without its Zipf bias.
+
 Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on a
 bounded sample of the same workload instead (rank 0 only).
 """
@@ -20,6 +26,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import gc
 import json
 import os
 import statistics
@@ -35,8 +42,13 @@ sys.path.insert(0, ROOT)
 
 from routing_dispatch_expert_fp32_b200 import workloads as wl  # noqa: E402
 
-DEFAULT_WORKLOAD = "skewed_drops"
+DEFAULT_WORKLOAD = "fine_grained"
+# Peaks used when MEASURED_PEAKS.json is absent (an earlier measurement on this
+# kind of B200: STREAM-style copy, cuBLAS bf16 burst and power-capped loop).
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# A timed region this long, or one that saw the power cap, is judged against
+# the sustained tensor peak; a shorter one at full clocks against the burst peak.
+SUSTAINED_REGION_MS = 1000.0
 
 
 def parse():
@@ -61,8 +73,10 @@ def parse():
                          "GEMM's rows (no dispatch pass); bf16 expert layers only")
     ap.add_argument("--no-graph", action="store_true",
                     help="issue the step kernel by kernel instead of replaying a CUDA graph")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other workloads, the backward and the f2/f4 timings")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
-                    help="target CPU time of the oracle sample (0: skip the CPU leg)")
+                    help="target CPU time of each oracle sample (0: skip the CPU legs)")
     return ap.parse_args()
 
 
@@ -83,11 +97,22 @@ def default_steps(w: wl.Workload) -> int:
             "fine_grained": 300, "bw_sweep": 1000}[w.name]
 
 
+# the other workloads of the one-rank line: (label, workload, timed steps)
+EXTRA_WORKLOADS = [
+    ("multistep_window", wl.WORKLOADS["multistep_window"], 96),
+    ("bw_sweep_T65536_zipf1.5", wl.WORKLOADS["bw_sweep"], 100),
+    ("bw_sweep_T65536_no_bias", wl.WORKLOADS["bw_sweep"].with_(zipf_s=None), 100),
+]
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
-            return json.load(f), "measured"
+            p = json.load(f)
+        out = dict(FALLBACK_PEAKS)
+        out.update({k: float(p[k]) for k in FALLBACK_PEAKS if k in p})
+        return out, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
 
 
@@ -127,38 +152,102 @@ def config_of(w: wl.Workload, n: int, fused: bool = False):
         c["experts"] = "identity"
     if w.steps > 1:
         c["popularity_window"] = w.W
+        c["batches"] = w.steps
     c["path"] = "fused" if fused else "unfused"
     return c
 
 
 # --------------------------------------------------------------- clocks ---
-class ClockSampler:
-    """nvidia-smi samples during the timed region (reads only)."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+REJECTING = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
-    def __init__(self, index: int):
-        self.index, self.proc, self.lines = index, None, []
+
+class ClockSampler:
+    """SM clock, throttle reasons and power read (query only) during a timed
+    region: NVML from a side thread at about 1-2 kHz, else nvidia-smi every
+    200 ms."""
+
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.nvml = None
+        self.samples = []
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(cuda_index).uuid)
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-")
+                                                     else "GPU-" + uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+            self.nvml, self.handle = pynvml, h
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.nvml = None
+
+    # -- NVML thread
+    def _loop(self):
+        nv, h = self.nvml, self.handle
+        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = reasons_fn(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((time.perf_counter(), float(sm), int(rs), pw))
+            except Exception:
+                pass
+            time.sleep(0.0003)
 
     def start(self):
+        self.samples = []
+        self.t0 = time.perf_counter()
+        if self.nvml is not None:
+            self.old_switch = sys.getswitchinterval()
+            sys.setswitchinterval(1e-4)
+            self.stop_flag = threading.Event()
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+            return
+        self.proc = None
         try:
+            q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                 "clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-i", str(self.index), "-lms", "200"],
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.cuda_index), "-lms", "200"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.lines = []
+            self.thread = threading.Thread(
+                target=lambda: [self.lines.append(x.strip()) for x in self.proc.stdout],
+                daemon=True)
             self.thread.start()
         except (OSError, ValueError):
             self.proc = None
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        dt = time.perf_counter() - self.t0
+        if self.nvml is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=2)
+            sys.setswitchinterval(self.old_switch)
+            sm = [s[1] for s in self.samples]
+            bits = 0
+            for s in self.samples:
+                bits |= s[2]
+            reasons = sorted(n for n, b in REASON_BITS.items() if bits & b)
+            return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                    "sm_min_mhz": min(sm) if sm else None, "reasons": reasons,
+                    "samples": len(sm), "rate_hz": round(len(sm) / dt, 1) if dt > 0 else None,
+                    "power_w_max": max(s[3] for s in self.samples) if sm else None,
+                    "source": "nvml"}
+        if getattr(self, "proc", None) is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -169,28 +258,44 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.lines:
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 7:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-                power.append(float(f[3]))
+                sm.append(float(f[0]))
+                mx = float(f[1])
+                power.append(float(f[2]))
             except ValueError:
                 continue
-            for name, v in zip(names, f[5:9]):
+            for name, v in zip(names, f[3:7]):
                 if v.lower() == "active":
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
                 "reasons": sorted(reasons), "samples": len(sm),
-                "power_w_max": max(power) if power else None}
+                "power_w_max": max(power) if power else None, "source": "nvidia-smi"}
+
+
+def tensor_peak(peaks, src, clocks, region_ms):
+    """The bf16 peak a tensor-bound kernel is judged against: the sustained one
+    for a region of a second or more or one that saw the power cap, else the
+    burst one."""
+    capped = clocks is not None and "sw_power_cap" in clocks.get("reasons", [])
+    key = "bf16_tflops_sustained" if (capped or region_ms >= SUSTAINED_REGION_MS) \
+        else "bf16_tflops"
+    why = ("power cap seen in the region" if capped else
+           f"region {region_ms:.0f} ms >= {SUSTAINED_REGION_MS:.0f} ms"
+           if region_ms >= SUSTAINED_REGION_MS else
+           f"region {region_ms:.0f} ms at full clocks")
+    return peaks[key], f"of {src} {key} ({why})"
 
 
 # ----------------------------------------------------------- reference ---
-def cpu_oracle_run(w: wl.Workload, target_s: float):
+def cpu_oracle_run(w: wl.Workload, target_s: float, parallel: bool = False):
     """The oracle as it stands on a bounded token sample of the workload:
-    gate, route (capacity rescaled to the sample), dispatch, FFN, combine."""
+    gate, route (capacity rescaled to the sample), dispatch, FFN, combine.
+    ``parallel`` uses the OpenMP build on every host core."""
     import oracle
 
+    cores = oracle.use_parallel(parallel)
     weights = wl.make_weights(w)
     inp = wl.make_step(w, 0)
 
@@ -217,7 +322,8 @@ def cpu_oracle_run(w: wl.Workload, target_s: float):
     if dt < target_s and n < w.T:
         n = min(w.T, max(n + 1, int(n * target_s / max(dt, 1e-6))))
         dt = run(n)
-    return n / dt, n, dt
+    oracle.use_parallel(False)
+    return n / dt, n, dt, cores
 
 
 def reference_arm(args, w):
@@ -226,11 +332,10 @@ def reference_arm(args, w):
         return
     steps = args.steps or 3
     times = []
-    n = 0
-    rate = 0.0
+    n, cores = 0, 1
     per = args.cpu_seconds / max(1, steps)
     for _ in range(steps):
-        rate, n, dt = cpu_oracle_run(w, per)
+        _, n, dt, cores = cpu_oracle_run(w, per, parallel=True)
         times.append(dt)
     value = n * len(times) / sum(times)
     line = {"impl": "reference", "metric": "MoE layer tokens/s", "value": value,
@@ -238,8 +343,9 @@ def reference_arm(args, w):
             "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
             "data": "synthetic", "config": config_of(w, args.gpus),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": f"first {n} tokens of the batch per step, whole layer"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"first {n} tokens of the batch per step, whole layer, "
+                                       f"OpenMP build on {cores} host threads"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -310,28 +416,38 @@ def backward_extras(moe, w, layer, b, weights, stream, torch, reps=20):
     return out
 
 
-def main():
-    args = parse()
-    w = workload_of(args)
-    if args.impl == "reference":
-        reference_arm(args, w)
-        return
-
+def max_over_ranks(dist, ms: float, device) -> float:
+    """The slowest rank's time (every rank gets it)."""
     import torch
-    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
-    from routing_dispatch_expert_fp32_b200 import moe
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    steps = args.steps or default_steps(w)
-    warmup = max(3, args.warmup)
+class Ctx:
+    """The process's torch, binding and rank layout."""
 
+    def __init__(self, torch, dist, moe, world, rank, local, args, peaks, peak_src):
+        self.torch, self.dist, self.moe = torch, dist, moe
+        self.world, self.rank, self.local = world, rank, local
+        self.args, self.peaks, self.peak_src = args, peaks, peak_src
+        self.hook = (lambda c: dist.all_reduce(c)) if world > 1 else None
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max_over_ranks(self, ms: float) -> float:
+        return ms if self.world == 1 else max_over_ranks(self.dist, ms, "cuda")
+
+
+def measure(ctx: Ctx, w: wl.Workload, steps: int, warmup: int, full: bool):
+    """Times `steps` layer steps of workload w (graph replay on one rank) and a
+    stage-by-stage pass; with `full` also the end-to-end path, the backward and
+    the f2/f4 kernels.  Returns the fields of the JSON line."""
+    torch, moe, args = ctx.torch, ctx.moe, ctx.args
+    world, rank = ctx.world, ctx.rank
+    peaks = ctx.peaks
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     to_dev = lambda a: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)  # noqa: E731
                         if a.dtype == np.uint16 else torch.from_numpy(a)).cuda()
@@ -343,12 +459,11 @@ def main():
     for s in range(nb):
         inp = wl.make_step(w, s, rank)
         batches.append({k: (None if v is None else to_dev(v)) for k, v in inp.items()})
+    fused = args.path == "fused"
     layer = moe.MoELayer(w.T, w.d, w.E, w.k, w.F, tdt, capacity=w.capacity, W=w.W, P=w.P,
-                         identity_experts=w.identity_experts, fused=args.path == "fused")
+                         identity_experts=w.identity_experts, fused=fused)
     stream = torch.cuda.current_stream()
-    hook = None
-    if world > 1:
-        hook = lambda c: dist.all_reduce(c)  # noqa: E731  global popularity (sum over ranks)
+    hook = ctx.hook
 
     def step(i, ev=None, collective=True):
         b = batches[i % nb]
@@ -390,20 +505,28 @@ def main():
     for i in range(nb):
         step(i)
         R_of.append(int(layer.offsets[-1].item()))
-    # One CUDA graph per input batch (single rank; multi-rank steps hold an
-    # NCCL call and are issued kernel by kernel).
-    use_graph = world == 1 and not args.no_graph
+    # CUDA graphs per input batch: one graph of the whole step on one rank; with
+    # several ranks two graphs (gate + route, the rest) around the NCCL
+    # all_reduce of the counts.
+    use_graph = not args.no_graph
     graphs = []
     if use_graph:
         for b in batches:
-            graphs.append(layer.capture(b["x"], weights.get("Wg"), weights.get("W1"),
-                                        weights.get("W2"), b["bias"], logits=b.get("logits")))
+            call = dict(x=b["x"], Wg=weights.get("Wg"), W1=weights.get("W1"),
+                        W2=weights.get("W2"), bias=b["bias"], logits=b.get("logits"))
+            graphs.append(layer.capture(**call) if world == 1 else
+                          layer.capture_split(**call, counts_hook=hook))
 
     def run_step(i):
-        if use_graph:
+        if not use_graph:
+            step(i)
+        elif world == 1:
             graphs[i % nb].replay()
         else:
-            step(i)
+            g_route, g_rest = graphs[i % nb]
+            g_route.replay()
+            hook(layer.counts)
+            g_rest.replay()
 
     # Concurrent batches (single rank, graphs): `conc` layer instances with
     # their own buffers and one shared popularity window; group g runs
@@ -414,14 +537,13 @@ def main():
             conc = 2
         else:
             conc = 3 if 4.0 * w.T * w.k * w.d * w.F < 2e11 else 1
-    conc = conc if use_graph else 1
+    conc = conc if use_graph and world == 1 else 1
     layers = [layer]
-    groups, group_batches = [], []
+    groups = []
     if conc > 1:
         for _ in range(conc - 1):
             extra = moe.MoELayer(w.T, w.d, w.E, w.k, w.F, tdt, capacity=w.capacity, W=w.W,
-                                 P=w.P, identity_experts=w.identity_experts,
-                                 fused=args.path == "fused")
+                                 P=w.P, identity_experts=w.identity_experts, fused=fused)
             extra.share_popularity(layer)
             layers.append(extra)
         for g in range(max(1, nb // conc)):
@@ -430,7 +552,6 @@ def main():
                           W2=weights.get("W2"), bias=batches[j]["bias"],
                           logits=batches[j].get("logits")) for j in idx]
             groups.append(moe.capture_concurrent(layers, calls))
-            group_batches.append(idx)
 
     def run_group(g):
         groups[g % len(groups)].replay()
@@ -442,13 +563,9 @@ def main():
             run_step(i)
     torch.cuda.synchronize()
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
     # ---- timed region: the step as shipped (graph replay), events on the stream ----
-    sampler = ClockSampler(local) if rank == 0 else None
-    barrier()
+    sampler = ClockSampler(ctx.local) if rank == 0 else None
+    ctx.barrier()
     torch.cuda.synchronize()
     if sampler:
         sampler.start()
@@ -466,12 +583,8 @@ def main():
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    ctx.barrier()
+    elapsed_ms = ctx.max_over_ranks(t_start.elapsed_time(t_end))
     # one batch at a time (the single-stream graphs), for comparison
     seq = None
     if conc > 1:
@@ -492,18 +605,151 @@ def main():
     stage_steps = min(steps, 500)
     nev = 6
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(stage_steps)]
-    barrier()
+    ctx.barrier()
     torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
     for i in range(stage_steps):
         step(i, evs[i])
     torch.cuda.synchronize()
-    barrier()
+    stage_clocks = sampler.stop() if sampler else None
+    ctx.barrier()
     stage_ms = np.zeros(nev - 1)
     for e in evs:
         stage_ms += np.array([e[j].elapsed_time(e[j + 1]) for j in range(nev - 1)])
+    stage_total_ms = float(stage_ms.sum())
     stage_ms /= stage_steps
 
+    out = {"elapsed_ms": elapsed_ms, "steps": steps,
+           "value": w.T * steps * world / (elapsed_ms * 1e-3),
+           "ms_per_step": elapsed_ms / steps, "clocks": clocks,
+           "gpu_launches": layer.launches_per_forward(gate=not w.logits_direct) * steps,
+           "timing": {"value": (f"CUDA-graph replay, {conc} independent batches in flight "
+                                "(one stream each, popularity updates in order)")
+                      if conc > 1 else "CUDA-graph replay of the whole step"
+                      if use_graph and world == 1 else
+                      "CUDA-graph replays of gate + route and of the rest of the step around "
+                      "the NCCL all_reduce of the counts" if use_graph else
+                      "kernels issued one by one (programmatic dependent launch)",
+                      "batches_in_flight": conc, "one_batch_at_a_time": seq,
+                      "stages_and_roofline": f"{stage_steps} steps issued stage by stage, "
+                                             "events between stages",
+                      "stage_clocks": stage_clocks}}
+
     # ---- end to end: pinned host x -> device, layer, y -> pinned host ----
+    if full:
+        out.update(e2e_measure(ctx, w, steps, nb, batches, weights, layer, layers, conc,
+                               use_graph, tdt))
+
+    # ---- next-row kernels: cross-layer correlation + popularity forecast ----
+    # Batches 0 and 1 stand for two consecutive layers of the same tokens.
+    extras = {}
+    if full and rank == 0 and not args.no_extras:
+        extras = f2_f4_backward_extras(ctx, w, step, nb, batches, weights, layer, stream)
+    out["extras"] = extras
+    out["device_error_bits"] = moe.moe_device_error()
+
+    # ---- per-stage numbers and the dominant kernel's roofline ----
+    R_mean = float(np.mean([R_of[i % nb] for i in range(stage_steps)]))
+    names = ["gate", "route+popularity", "dispatch", "expert_ffn", "combine"]
+    es = 2 if w.dtype == "bf16" else 4
+    per = {}
+    alg = {
+        "gate": (2.0 * w.T * w.d * w.E, "flop") if not w.logits_direct else (0, "flop"),
+        "route+popularity": (w.T * w.E * 4 + w.T * w.k * 4 * 4 + R_mean * 4, "byte"),
+        "dispatch": ((0 if layer.fused else w.T * w.d * es + R_mean * w.d * es
+                      + w.T * w.k * 4), "byte"),
+        "expert_ffn": (4.0 * R_mean * w.d * w.F, "flop"),
+        "combine": (R_mean * w.d * es + w.T * w.d * es + w.T * w.k * 8, "byte"),
+    }
+    tc_peak, tc_src = tensor_peak(peaks, ctx.peak_src, stage_clocks, stage_total_ms)
+    for j, n in enumerate(names):
+        amount, kind = alg[n]
+        ms = float(stage_ms[j])
+        ent = {"ms": ms}
+        if ms > 0 and amount:
+            if kind == "flop":
+                ent["tflops"] = amount / (ms * 1e-3) / 1e12
+                ent["frac_bf16"] = ent["tflops"] / tc_peak
+            else:
+                ent["gbs"] = amount / (ms * 1e-3) / 1e9
+                ent["frac_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
+        per[n] = ent
+    out["stages"] = per
+    out["R_mean"] = R_mean
+    if w.identity_experts:
+        dom = "dispatch" if per["dispatch"]["ms"] >= per["combine"]["ms"] else "combine"
+        amount = alg[dom][0]
+        roof = {"bound": "hbm", "kernel": f"{dom}_kernel",
+                "achieved": amount / (per[dom]["ms"] * 1e-3) / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "peak_source": f"of {ctx.peak_src} hbm_gbs",
+                "bytes_per_launch": amount}
+    else:
+        # the grouped GEMM: two launches per step, 2*R*d*F flops each
+        launch_ms = per["expert_ffn"]["ms"] / 2
+        # the library's rule: R_max / E >= 1024 (dense): 2-CTA pair tiles for
+        # the whole 256-row blocks of every group, then 1-CTA tiles for the
+        # tails; else pair tiles when 128-row tiles would fill fewer than three
+        # waves of SMs, else 1-CTA tiles
+        nsm = torch.cuda.get_device_properties(ctx.local).multi_processor_count
+
+        def kernel_for(N):
+            if w.dtype != "bf16" or layer.fused:
+                return "gemm_tc_kernel"
+            if w.T * w.k >= 1024 * w.E:
+                return "gemm_tc2_kernel+gemm_tc_kernel"
+            tiles = (w.T * w.k // 128 + w.E) * ((N + 255) // 256)
+            return "gemm_tc2_kernel" if tiles < 3 * nsm else "gemm_tc_kernel"
+        kinds = [kernel_for(N) for N in (w.F, w.d)]
+        achieved = 2.0 * R_mean * w.d * w.F / (launch_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": kinds[0] if kinds[0] == kinds[1]
+                else " | ".join(kinds), "achieved": achieved, "peak": tc_peak,
+                "unit": "TFLOP/s", "peak_source": tc_src,
+                "frac_burst": achieved / peaks["bf16_tflops"],
+                "frac_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "flops_per_launch": 2.0 * R_mean * w.d * w.F}
+        # mixed bound of the grouped GEMM: every expert's weights are read once
+        # per launch (E*d*F*s bytes) besides the rows; experts with few rows
+        # are bound by that stream, not by the tensor cores
+        weight_bytes = w.E * w.d * w.F * es
+        act_bytes = R_mean * (w.d + w.F) * es
+        t_hbm = (weight_bytes + act_bytes) / (peaks["hbm_gbs"] * 1e9) * 1e3
+        t_tc = 2.0 * R_mean * w.d * w.F / (tc_peak * 1e12) * 1e3
+        roof["mixed_bound"] = {
+            "hbm_ms_per_launch": t_hbm, "tensor_ms_per_launch": t_tc,
+            "binding": "hbm" if t_hbm > t_tc else "tensor",
+            "frac_of_binding": max(t_hbm, t_tc) / launch_ms,
+            "note": "weights E*d*F*s + rows R*(d+F)*s bytes per launch at the HBM peak vs "
+                    "2*R*d*F flops at the tensor peak"}
+        if w.dtype == "f32":
+            # fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x the max SM clock
+            roof["bound"] = "alu"
+            roof["kernel"] = "gemm_simt_f32_kernel"
+            roof["peak"] = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+            roof["peak_source"] = "derived fp32 FMA peak: 148 x 128 x 2 x sm_max_mhz"
+            roof.pop("frac_burst", None)
+            roof.pop("frac_sustained", None)
+            roof.pop("mixed_bound", None)
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = (gemm_traffic(w.name + ("/fused" if layer.fused else ""), roof["kernel"])
+                       if roof["kernel"].startswith("gemm_tc") and args.tokens == 0
+                       and args.experts == 0 else None)
+    out["roofline"] = roof
+
+    # release this workload's device memory before the next one
+    del graphs, groups, layers, layer, batches, weights
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def e2e_measure(ctx, w, steps, nb, batches, weights, layer, layers, conc, use_graph, tdt):
+    """The same steps through the public API with every batch's x (and logits)
+    copied in from pinned host memory and y copied back, inside the timed region."""
+    torch, moe, hook = ctx.torch, ctx.moe, ctx.hook
+    stream = torch.cuda.current_stream()
     e2e_steps = max(10, steps // 4)
     host_x = [batches[i]["x"].cpu().pin_memory() for i in range(nb)]
     host_logits = [None if batches[i].get("logits") is None else
@@ -524,8 +770,7 @@ def main():
                       logits=dlog, counts_hook=hook)
         host_y.copy_(layer.y, non_blocking=True)
 
-    e2e_pipelined = use_graph
-    if e2e_pipelined:
+    if use_graph and ctx.world == 1:
         # Two units, each a graph over `conc` batches with its own layer
         # instances and device input buffers; copies run on their own streams
         # so unit u's inputs arrive and unit u-1's outputs leave while the
@@ -549,8 +794,7 @@ def main():
         second = []
         for _ in range(conc):
             extra = moe.MoELayer(w.T, w.d, w.E, w.k, w.F, tdt, capacity=w.capacity, W=w.W,
-                                 P=w.P, identity_experts=w.identity_experts,
-                                 fused=args.path == "fused")
+                                 P=w.P, identity_experts=w.identity_experts, fused=layer.fused)
             extra.share_popularity(layer)
             second.append(extra)
         units = [make_unit(layers, 0), make_unit(second, conc % nb)]
@@ -590,10 +834,13 @@ def main():
             e2e_unit(it)
         e1.record(s_out)
         torch.cuda.synchronize()
+        note = ("pinned host x in and y out every step, on copy streams that overlap the other "
+                "of two alternating graph units")
+        del units, second
     else:
         for i in range(3):
             e2e_step(i)
-        barrier()
+        ctx.barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -601,159 +848,135 @@ def main():
             e2e_step(i)
         e1.record(stream)
         torch.cuda.synchronize()
-        barrier()
-    e2e_ms = e0.elapsed_time(e1)
+        ctx.barrier()
+        note = "pinned host x in and y out every step, in stream order"
+    e2e_ms = ctx.max_over_ranks(e0.elapsed_time(e1))
+    return {"e2e": {"value": w.T * e2e_steps * ctx.world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "note": note}}
+
+
+def f2_f4_backward_extras(ctx, w, step, nb, batches, weights, layer, stream):
+    torch, moe = ctx.torch, ctx.moe
+    ids_a = torch.empty_like(layer.ids)
+    step(0, collective=False)  # rank 0 only: no collective here
+    ids_a.copy_(layer.ids)
+    step(1 % nb, collective=False)
+    C = torch.zeros(w.E, w.E, dtype=torch.int32, device="cuda")
+    pred = torch.empty(w.E, device="cuda")
+    hot_f = torch.empty(max(w.P, 1), dtype=torch.int32, device="cuda")
+    reps = 200
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for _ in range(3):
+        moe.moe_correlation_update(ids_a, layer.ids, C)
+        moe.moe_popularity_forecast(layer.mean, C, w.k, w.k, pred, w.P, hot_f)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(reps):
+        moe.moe_correlation_update(ids_a, layer.ids, C)
+    ev[1].record(stream)
+    for _ in range(reps):
+        moe.moe_popularity_forecast(layer.mean, C, w.k, w.k, pred, w.P, hot_f)
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    corr_ms = ev[0].elapsed_time(ev[1]) / reps
+    fc_ms = ev[1].elapsed_time(ev[2]) / reps
+    # GShard balancing loss of the last routing call (re-reads the logits)
+    logits_last = batches[1 % nb].get("logits")
+    if logits_last is None:
+        logits_last = layer.logits
+    aux_loss = torch.empty(1, device="cuda")
+    aux_P = torch.empty(w.E, device="cuda")
+    bias_last = batches[1 % nb]["bias"]
+    for _ in range(3):
+        moe.moe_aux_loss(logits_last, bias_last, w.k, layer.counts, aux_loss, aux_P,
+                         layer.workspace)
+    ev[0].record(stream)
+    for _ in range(reps):
+        moe.moe_aux_loss(logits_last, bias_last, w.k, layer.counts, aux_loss, aux_P,
+                         layer.workspace)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    aux_ms = ev[0].elapsed_time(ev[1]) / reps
+    corr_bytes = 2 * w.T * w.k * 4 + 2 * w.E * w.E * 4
+    bwd = (None if layer.fused else
+           backward_extras(moe, w, layer, batches[1 % nb], weights, stream, torch))
+    return {
+        "backward": bwd,
+        "correlation_update": {"ms": corr_ms, "pairs": w.T * w.k * w.k,
+                               "gbs": corr_bytes / (corr_ms * 1e-3) / 1e9},
+        "popularity_forecast": {"ms": fc_ms, "E": w.E},
+        "aux_loss": {"ms": aux_ms, "value": float(aux_loss.item()),
+                     "gbs": w.T * w.E * 4 / (aux_ms * 1e-3) / 1e9},
+        "note": "timed separately (200 back-to-back launches each), outside the step",
+    }
+
+
+def workload_summary(w, m):
+    """The compact entry of one extra workload in the line."""
+    return {"config": config_of(w, 1), "value": m["value"], "unit": "tokens/s",
+            "ms_per_step": m["ms_per_step"], "steps": m["steps"], "R_mean": m["R_mean"],
+            "roofline": m["roofline"], "stages": m["stages"], "clocks": m["clocks"],
+            "stage_clocks": m["timing"]["stage_clocks"],
+            "batches_in_flight": m["timing"]["batches_in_flight"],
+            "one_batch_at_a_time": m["timing"]["one_batch_at_a_time"],
+            "device_error_bits": m["device_error_bits"]}
+
+
+def main():
+    args = parse()
+    w = workload_of(args)
+    if args.impl == "reference":
+        reference_arm(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from routing_dispatch_expert_fp32_b200 import moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
     if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    # ---- next-row kernels: cross-layer correlation + popularity forecast ----
-    # Batches 0 and 1 stand for two consecutive layers of the same tokens.
-    extras = {}
-    if rank == 0:
-        ids_a = torch.empty_like(layer.ids)
-        step(0, collective=False)  # rank 0 only: no collective here
-        ids_a.copy_(layer.ids)
-        step(1 % nb, collective=False)
-        C = torch.zeros(w.E, w.E, dtype=torch.int32, device="cuda")
-        pred = torch.empty(w.E, device="cuda")
-        hot_f = torch.empty(max(w.P, 1), dtype=torch.int32, device="cuda")
-        reps = 200
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        for _ in range(3):
-            moe.moe_correlation_update(ids_a, layer.ids, C)
-            moe.moe_popularity_forecast(layer.mean, C, w.k, w.k, pred, w.P, hot_f)
-        torch.cuda.synchronize()
-        ev[0].record(stream)
-        for _ in range(reps):
-            moe.moe_correlation_update(ids_a, layer.ids, C)
-        ev[1].record(stream)
-        for _ in range(reps):
-            moe.moe_popularity_forecast(layer.mean, C, w.k, w.k, pred, w.P, hot_f)
-        ev[2].record(stream)
-        torch.cuda.synchronize()
-        corr_ms = ev[0].elapsed_time(ev[1]) / reps
-        fc_ms = ev[1].elapsed_time(ev[2]) / reps
-        # GShard balancing loss of the last routing call (re-reads the logits)
-        logits_last = batches[1 % nb].get("logits")
-        if logits_last is None:
-            logits_last = layer.logits
-        aux_loss = torch.empty(1, device="cuda")
-        aux_P = torch.empty(w.E, device="cuda")
-        bias_last = batches[1 % nb]["bias"]
-        for _ in range(3):
-            moe.moe_aux_loss(logits_last, bias_last, w.k, layer.counts, aux_loss, aux_P,
-                             layer.workspace)
-        ev[0].record(stream)
-        for _ in range(reps):
-            moe.moe_aux_loss(logits_last, bias_last, w.k, layer.counts, aux_loss, aux_P,
-                             layer.workspace)
-        ev[1].record(stream)
-        torch.cuda.synchronize()
-        aux_ms = ev[0].elapsed_time(ev[1]) / reps
-        corr_bytes = 2 * w.T * w.k * 4 + 2 * w.E * w.E * 4
-        bwd = (None if layer.fused else
-               backward_extras(moe, w, layer, batches[1 % nb], weights, stream, torch))
-        extras = {
-            "backward": bwd,
-            "correlation_update": {"ms": corr_ms, "pairs": w.T * w.k * w.k,
-                                   "gbs": corr_bytes / (corr_ms * 1e-3) / 1e9},
-            "popularity_forecast": {"ms": fc_ms, "E": w.E},
-            "aux_loss": {"ms": aux_ms, "value": float(aux_loss.item()),
-                         "gbs": w.T * w.E * 4 / (aux_ms * 1e-3) / 1e9},
-            "note": "timed separately (200 back-to-back launches each), outside the step",
-        }
-    dev_err = moe.moe_device_error()
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    peaks, peak_src = load_peaks()
+    ctx = Ctx(torch, dist, moe, world, rank, local, args, peaks, peak_src)
+    steps = args.steps or default_steps(w)
+    warmup = max(3, args.warmup)
+
+    head = measure(ctx, w, steps, warmup, full=True)
+    extras = head.pop("extras")
+    headline_default = (args.workload == DEFAULT_WORKLOAD and not args.tokens
+                        and not args.no_bias and not args.experts and args.path == "unfused")
+    if world == 1 and headline_default and not args.no_extras:
+        extras["workloads"] = {}
+        for label, w2, st in EXTRA_WORKLOADS:
+            extras["workloads"][label] = workload_summary(w2, measure(ctx, w2, st, warmup,
+                                                                      full=False))
 
     if rank == 0:
-        peaks, peak_src = load_peaks()
-        R_mean = float(np.mean([R_of[i % nb] for i in range(stage_steps)]))
-        names = ["gate", "route+popularity", "dispatch", "expert_ffn", "combine"]
-        es = 2 if w.dtype == "bf16" else 4
-        per = {}
-        alg = {
-            "gate": (2.0 * w.T * w.d * w.E, "flop") if not w.logits_direct else (0, "flop"),
-            "route+popularity": (w.T * w.E * 4 + w.T * w.k * 4 * 4 + R_mean * 4, "byte"),
-            "dispatch": ((0 if layer.fused else w.T * w.d * es + R_mean * w.d * es
-                          + w.T * w.k * 4), "byte"),
-            "expert_ffn": (4.0 * R_mean * w.d * w.F, "flop"),
-            "combine": (R_mean * w.d * es + w.T * w.d * es + w.T * w.k * 8, "byte"),
-        }
-        for j, n in enumerate(names):
-            amount, kind = alg[n]
-            ms = float(stage_ms[j])
-            ent = {"ms": ms}
-            if ms > 0 and amount:
-                if kind == "flop":
-                    ent["tflops"] = amount / (ms * 1e-3) / 1e12
-                    ent["frac_bf16_sustained"] = ent["tflops"] / peaks["bf16_tflops_sustained"]
-                else:
-                    ent["gbs"] = amount / (ms * 1e-3) / 1e9
-                    ent["frac_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
-            per[n] = ent
-        if w.identity_experts:
-            dom = "dispatch" if per["dispatch"]["ms"] >= per["combine"]["ms"] else "combine"
-            amount = alg[dom][0]
-            roof = {"bound": "hbm", "kernel": f"{dom}_kernel",
-                    "achieved": amount / (per[dom]["ms"] * 1e-3) / 1e9,
-                    "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-        else:
-            # the grouped GEMM: two launches per step, 2*R*d*F flops each
-            launch_ms = per["expert_ffn"]["ms"] / 2
-            # the library takes 2-CTA pair tiles when R_max / E >= 1024 or when
-            # 128-row tiles would fill fewer than three waves of SMs
-            nsm = torch.cuda.get_device_properties(local).multi_processor_count
-
-            def pair_for(N):
-                tiles = (w.T * w.k // 128 + w.E) * ((N + 255) // 256)
-                return (w.dtype == "bf16" and not layer.fused
-                        and (w.T * w.k >= 1024 * w.E or tiles < 3 * nsm))
-            kinds = ["gemm_tc2_kernel" if pair_for(N) else "gemm_tc_kernel" for N in (w.F, w.d)]
-            roof = {"bound": "tensor", "kernel": kinds[0] if kinds[0] == kinds[1]
-                    else "+".join(kinds),
-                    "achieved": 2.0 * R_mean * w.d * w.F / (launch_ms * 1e-3) / 1e12,
-                    "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
-            if w.dtype == "f32":
-                # fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x the max SM clock
-                roof["bound"] = "alu"
-                roof["kernel"] = "gemm_simt_f32_kernel"
-                roof["peak"] = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["peak_source"] = (
-            "derived fp32 FMA peak: 148 x 128 x 2 x sm_max_mhz" if roof["bound"] == "alu" else
-            f"{peak_src} ({'bf16_tflops_sustained' if roof['unit'] == 'TFLOP/s' else 'hbm_gbs'})")
-        roof["traffic"] = (gemm_traffic(w.name + ("/fused" if layer.fused else ""), roof["kernel"])
-                           if roof["kernel"].startswith("gemm_tc") and args.tokens == 0
-                           and args.experts == 0 else None)
-        value = w.T * steps * world / (elapsed_ms * 1e-3)
         cpu = None
         if world == 1 and args.cpu_seconds > 0:
-            rate, n, dt = cpu_oracle_run(w, args.cpu_seconds)
-            cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                   "sample": f"first {n} tokens of one batch through the whole layer "
-                             f"({dt:.1f} s, capacity rescaled to the sample)"}
-        line = {"metric": "MoE layer tokens/s", "value": value, "unit": "tokens/s",
+            rate_all, n_all, dt_all, cores = cpu_oracle_run(w, args.cpu_seconds, parallel=True)
+            rate_1, n_1, dt_1, _ = cpu_oracle_run(w, args.cpu_seconds, parallel=False)
+            cpu = {"value": rate_all, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                   "sample": f"first {n_all} tokens of one batch through the whole layer "
+                             f"({dt_all:.1f} s, capacity rescaled to the sample), OpenMP build "
+                             f"on {cores} host threads",
+                   "one_core": {"value": rate_1, "unit": "tokens/s", "cores": 1,
+                                "sample": f"first {n_1} tokens ({dt_1:.1f} s), "
+                                          "single-threaded build"}}
+        line = {"metric": "MoE layer tokens/s", "value": head["value"], "unit": "tokens/s",
                 "n_gpus": world, "steps": steps, "warmup": warmup,
-                "ms_per_step": elapsed_ms / steps, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-                "config": config_of(w, world, layer.fused),
-                "e2e": {"value": w.T * e2e_steps * world / (e2e_ms * 1e-3), "unit": "tokens/s",
-                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                        "note": ("pinned host x in and y out every step, on copy streams that "
-                                 "overlap the other of two alternating graph units"
-                                 if e2e_pipelined else
-                                 "pinned host x in and y out every step, in stream order")},
-                "gpu_launches": layer.launches_per_forward(gate=not w.logits_direct) * steps,
-                "roofline": roof, "stages": per, "clocks": clocks, "cpu_baseline": cpu,
-                "timing": {"value": (f"CUDA-graph replay, {conc} independent batches in flight "
-                                     "(one stream each, popularity updates in order)")
-                           if conc > 1 else "CUDA-graph replay of the whole step" if use_graph
-                           else "kernels issued one by one (programmatic dependent launch)",
-                           "batches_in_flight": conc,
-                           "one_batch_at_a_time": seq,
-                           "stages_and_roofline": f"{stage_steps} steps issued stage by stage, "
-                                                  "events between stages"},
-                "extras": extras, "device_error_bits": dev_err}
+                "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+                "config": config_of(w, world, args.path == "fused"),
+                "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+                "roofline": head["roofline"], "stages": head["stages"],
+                "clocks": head["clocks"], "cpu_baseline": cpu, "timing": head["timing"],
+                "extras": extras, "device_error_bits": head["device_error_bits"]}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

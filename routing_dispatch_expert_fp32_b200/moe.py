@@ -282,15 +282,29 @@ class MoELayer:
 
     def forward(self, x, Wg=None, W1=None, W2=None, bias=None, logits=None, stream=None,
                 popularity=True, counts_hook=None, popularity_done=None):
+        """One layer step: ``forward_route``, then (when ``popularity``) the
+        counts hook -- e.g. an all_reduce of the per-expert counts across
+        data-parallel ranks -- and ``forward_rest``."""
+        self.forward_route(x, Wg, bias, logits, stream)
+        if popularity and counts_hook is not None:
+            counts_hook(self.counts)
+        return self.forward_rest(x, W1, W2, stream, popularity, popularity_done)
+
+    def forward_route(self, x, Wg=None, bias=None, logits=None, stream=None):
+        """Gate (unless logits are given) and route: the part of a step before
+        the per-expert counts may be exchanged."""
         if logits is None:
             moe_gate(x, Wg, self.logits, stream)
             logits = self.logits
         moe_route(logits, bias, self.k, self.capacity, self.ids, self.w, self.counts, self.kept,
                   self.offsets, self.slot_row, self.row_slot, self.n_dropped, self.workspace,
                   stream)
+
+    def forward_rest(self, x, W1=None, W2=None, stream=None, popularity=True,
+                     popularity_done=None):
+        """Popularity update, dispatch, expert FFN and combine (after
+        ``forward_route`` and any exchange of the counts); returns y."""
         if popularity:
-            if counts_hook is not None:  # e.g. an all_reduce of the counts across ranks
-                counts_hook(self.counts)
             moe_popularity_update_dev(self.counts, self.hist, self.step_dev, self.mean, self.P,
                                       self.hot, stream)
             if popularity_done is not None:
@@ -393,6 +407,25 @@ class MoELayer:
         with torch.cuda.graph(graph):
             self.forward(x, Wg, W1, W2, bias, logits=logits, popularity=popularity)
         return graph
+
+    def capture_split(self, x, Wg=None, W1=None, W2=None, bias=None, logits=None,
+                      counts_hook=None):
+        """Records one step as two CUDA graphs, (route, rest): gate + route, and
+        popularity + dispatch + expert FFN + combine.  A multi-rank step
+        replays the first, runs the counts exchange (``counts_hook``, e.g. an
+        NCCL all_reduce, outside any graph) and replays the second.  Capturing
+        runs one step (with the hook), which advances the popularity window."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.forward(x, Wg, W1, W2, bias, logits=logits, counts_hook=counts_hook)
+        torch.cuda.current_stream().wait_stream(side)
+        g_route, g_rest = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_route):
+            self.forward_route(x, Wg, bias, logits)
+        with torch.cuda.graph(g_rest):
+            self.forward_rest(x, W1, W2)
+        return g_route, g_rest
 
     def launches_per_forward(self, gate=True, popularity=True) -> int:
         """Kernel launches one forward makes (route is three kernels)."""

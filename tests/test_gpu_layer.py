@@ -212,3 +212,53 @@ def test_concurrent_batches_match_sequential_and_keep_one_window(moe):
     assert np.array_equal(host(layers[0].mean), mean_ref)
     assert np.array_equal(host(layers[0].hot)[: w.P], hot_ref)
     assert moe.moe_device_error() == 0
+
+
+def _expert_subset(offsets, rng, n_hot=4, n_cold=4, n_rand=8):
+    """The n_hot largest and n_cold smallest non-empty groups and n_rand others."""
+    sizes = np.diff(offsets)
+    nonempty = [int(e) for e in np.argsort(-sizes, kind="stable") if sizes[e] > 0]
+    pick = nonempty[:n_hot] + nonempty[-n_cold:]
+    rest = [e for e in nonempty if e not in pick]
+    pick += rng.choice(rest, min(n_rand, len(rest)), replace=False).tolist()
+    return sorted(set(pick))
+
+
+@pytest.mark.parametrize("name", ["multistep_window", "fine_grained"])
+def test_every_row_of_sixteen_experts_at_full_size(moe, name):
+    """Every expert-output row (H and Yp) of 16 experts -- the 4 hottest, the 4
+    coldest and 8 seeded others -- at the workload's full size, in the launch
+    configuration bench.py times, against the oracle (its OpenMP build on all
+    host cores), each expert on its own scale."""
+    w = wl.WORKLOADS[name]
+    weights = wl.make_weights(w)
+    inp = wl.make_step(w, 0)
+    layer = make_layer(moe, w)
+    dW = {k: dev(v) for k, v in weights.items()}
+    layer.forward(dev(inp["x"]), dW["Wg"], dW["W1"], dW["W2"], dev(inp["bias"]))
+    torch.cuda.synchronize()
+    assert moe.moe_device_error() == 0
+    offsets = host(layer.offsets)
+    row_slot = host(layer.row_slot)
+    # the routing itself is checked bit for bit by the single-step tests; here
+    # the grouped rows are taken as the GPU laid them out
+    experts = _expert_subset(offsets, np.random.default_rng(11))
+    assert len(experts) >= 16
+    rows = np.concatenate([np.arange(offsets[e], offsets[e + 1]) for e in experts])
+    expert_of_row = np.repeat(experts, [offsets[e + 1] - offsets[e] for e in experts])
+    rows_d = torch.from_numpy(rows).cuda()
+    H, Y = host(layer.H[rows_d]), host(layer.Yp[rows_d])
+    xr = inp["x"][row_slot[rows] // w.k]
+    try:
+        oracle.use_parallel(True)
+        Yr, Hr = oracle.expert_ffn_rows(xr, expert_of_row, weights["W1"], weights["W2"],
+                                        want_h=True)
+    finally:
+        oracle.use_parallel(False)
+    start = 0
+    for e in experts:
+        n = int(offsets[e + 1] - offsets[e])
+        sl = slice(start, start + n)
+        assert_close(H[sl], Hr[sl], f"H expert {e} ({n} rows)")
+        assert_close(Y[sl], Yr[sl], f"Yp expert {e} ({n} rows)")
+        start += n
