@@ -140,9 +140,11 @@ MOE_API int moe_route(const float* logits, const float* bias, int T, int E, int 
  * results and errors as moe_route, minus the workspace: the scratch is a
  * 4 MiB device array built into the library (held on every device that loads
  * it until the process exits).
- *  - Size limit: moe_route_workspace_size(T, E, k) <= 4 MiB (e.g. E = 256 up
- *    to T = 524032 tokens, E = 1024 up to T = 130816); larger problems return
- *    MOE_ERR_WORKSPACE and launch nothing.
+ *  - Size limit: the router's two per-chunk tables for chunks of 128 tokens,
+ *    2 * ceil(T / 128) * E int32 (each table rounded up to 256 bytes), plus
+ *    256 bytes must fit 4 MiB (e.g. E = 256 up to T = 262016 tokens, E = 1024
+ *    up to T = 65408); larger problems return MOE_ERR_WORKSPACE and launch
+ *    nothing.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
  *    before any stream capture.

@@ -9,15 +9,18 @@
 // torch.topk), so each of the k rounds picks an expert in [0, E) whatever the
 // input.  Equal keys go to the lower expert index.
 //
-// Three launches, no inter-CTA waiting (chunks of 256 tokens):
+// Three launches, no inter-CTA waiting (chunks of 128 tokens, or 64 / 32 when
+// that gives too few chunks to fill the GPU):
 //   K1 route_topk    one CTA per chunk.  E <= 32: one token per thread; the
 //                    row's keys sit in registers (16-byte loads when E % 4 == 0)
 //                    and k passes of an unrolled max pick the experts.  E > 32:
 //                    one token per warp, lane l holding experts
 //                    (i / V) * 32V + l * V + i % V (V-wide vector loads), with
-//                    the next tokens' logits loaded while the current one is
-//                    ranked; per round the largest key by a warp reduction, then
-//                    the lowest index among the lanes holding it.  Weights
+//                    the next tokens' logits loaded while the current ones are
+//                    ranked; a lane sorts its candidates once (up to 8 of them),
+//                    then per round the largest head key by a warp reduction,
+//                    the lowest index among the lanes holding it, and the owner
+//                    pops its head.  Weights
 //                    w_j = exp(z_j - z_0) / sum_i exp(z_i - z_0), the sum in rank
 //                    order.  Per-chunk expert histogram in shared memory
 //                    (atomicAdd on counts commutes: the result is order-free).
@@ -38,15 +41,28 @@
 
 namespace moe {
 
-constexpr int kChunk = 256;        // tokens per chunk (= per CTA in K1 and K3)
-constexpr int kThreads = kChunk;   // K3 (and K1 for E <= 32): one token per thread
-constexpr int kWarps = kThreads / 32;
+constexpr int kMaxChunk = 128;        // tokens per chunk at most (= per CTA in K1 and K3)
+constexpr int kMaxWarps = kMaxChunk / 32;
+constexpr int kChunkTarget = 296;     // chunks wanted: two per SM of a 148-SM B200
+
+// Tokens per chunk: 128, or 64 / 32 when 128 would leave fewer than
+// kChunkTarget chunks, so that smaller batches still spread over the GPU.  A
+// function of T alone (the workspace size depends on it).
+static int chunk_tokens(int T) {
+    if ((T + 127) / 128 >= kChunkTarget) return 128;
+    if ((T + 63) / 64 >= kChunkTarget) return 64;
+    return 32;
+}
 constexpr int kScanThreads = 1024;
 
-// K1 threads for E > 32: 32 warps of 8 tokens; 8 warps of 32 tokens when a
+// K1 threads for E > 32: 8 warps of 16 tokens; 4 warps of 32 tokens when a
 // lane holds 16 or more keys (register budget).
 template <int VPL>
-constexpr int warp_topk_threads() { return VPL >= 16 ? 256 : 1024; }
+constexpr int warp_topk_threads() { return VPL >= 16 ? 128 : 256; }
+// CTAs per SM the register budget is held to (four: every chunk of the
+// largest batches resident in one wave).
+template <int VPL>
+constexpr int warp_topk_min_blocks() { return VPL <= 4 ? 4 : (VPL <= 8 ? 3 : 1); }
 
 // Order key of z: larger z -> larger key; -0.0 ties with +0.0; NaN above all.
 // Keys of numbers are >= 0x007FFFFF (that of -inf), so 0 is free as "none".
@@ -64,10 +80,10 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 // rounds; vw (1, 2 or 4) is the load width (the host checks E % vw == 0 and the
 // alignment of `logits`).
 template <int EMAX, int KMAX>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kMaxChunk)
 route_topk_lane_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
-                       int E, int k, int vw, int32_t* __restrict__ ids, float* __restrict__ w,
-                       int32_t* __restrict__ chunk_hist, int32_t* err) {
+                       int E, int k, int vw, int ch, int32_t* __restrict__ ids,
+                       float* __restrict__ w, int32_t* __restrict__ chunk_hist, int32_t* err) {
     __shared__ int s_hist[EMAX];
     __shared__ float s_bias[EMAX];
     pdl_wait();
@@ -78,7 +94,7 @@ route_topk_lane_kernel(const float* __restrict__ logits, const float* __restrict
             (bias != nullptr && (int)threadIdx.x < E) ? bias[threadIdx.x] : 0.0f;
     }
     __syncthreads();
-    const int t = blockIdx.x * kChunk + threadIdx.x;
+    const int t = blockIdx.x * ch + threadIdx.x;  // blockDim.x == ch
     if (t < T) {
         const float* row = logits + (size_t)t * E;
         float z[EMAX];
@@ -148,6 +164,31 @@ route_topk_lane_kernel(const float* __restrict__ logits, const float* __restrict
 // E > 32: one token per warp; each lane holds VPL keys, loaded VW floats at a
 // time: slot i of lane l is expert (i / VW) * 32 * VW + l * VW + i % VW, which
 // grows with i, so a lane's strict '>' scan keeps the lowest index of a tie.
+// Sorts VPL (key, expert) pairs into (key desc, expert asc) order with a
+// fixed comparator network (Batcher's for 8, the optimal one for 4).
+__device__ __forceinline__ void cas_desc(uint32_t& ka, int& ea, uint32_t& kb, int& eb) {
+    const bool sw = kb > ka || (kb == ka && eb < ea);
+    const uint32_t k0 = sw ? kb : ka, k1 = sw ? ka : kb;
+    const int e0 = sw ? eb : ea, e1 = sw ? ea : eb;
+    ka = k0; kb = k1; ea = e0; eb = e1;
+}
+template <int VPL>
+__device__ __forceinline__ void sort_desc(uint32_t (&k)[VPL], int (&e)[VPL]) {
+    if constexpr (VPL == 2) {
+        cas_desc(k[0], e[0], k[1], e[1]);
+    } else if constexpr (VPL == 4) {
+        constexpr int net[5][2] = {{0, 1}, {2, 3}, {0, 2}, {1, 3}, {1, 2}};
+#pragma unroll
+        for (int c = 0; c < 5; ++c) cas_desc(k[net[c][0]], e[net[c][0]], k[net[c][1]], e[net[c][1]]);
+    } else if constexpr (VPL == 8) {
+        constexpr int net[19][2] = {{0, 1}, {2, 3}, {4, 5}, {6, 7}, {0, 2}, {1, 3}, {4, 6},
+                                    {5, 7}, {1, 2}, {5, 6}, {0, 4}, {1, 5}, {2, 6}, {3, 7},
+                                    {2, 4}, {3, 5}, {1, 2}, {3, 4}, {5, 6}};
+#pragma unroll
+        for (int c = 0; c < 19; ++c) cas_desc(k[net[c][0]], e[net[c][0]], k[net[c][1]], e[net[c][1]]);
+    }
+}
+
 template <int VPL, int VW>
 __device__ __forceinline__ void load_lane(const float* __restrict__ row, int lane_vw, int E,
                                           float (&v)[VPL]) {
@@ -169,15 +210,22 @@ __device__ __forceinline__ void load_lane(const float* __restrict__ row, int lan
 }
 
 template <int VPL, int VW>
-__global__ void __launch_bounds__(warp_topk_threads<VPL>())
+__global__ void __launch_bounds__(warp_topk_threads<VPL>(), warp_topk_min_blocks<VPL>())
 route_topk_warp_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
-                       int E, int k, int32_t* __restrict__ ids, float* __restrict__ w,
+                       int E, int k, int ch, int32_t* __restrict__ ids, float* __restrict__ w,
                        int32_t* __restrict__ chunk_hist, int32_t* err) {
     constexpr int kT = warp_topk_threads<VPL>();
-    constexpr int kPerWarp = kChunk / (kT / 32);           // tokens per warp
-    constexpr int D = VPL <= 4 ? 2 : 1;                    // tokens in flight per warp
-    static_assert(kPerWarp % D == 0, "token groups");
+    const int per_warp = ch / (kT / 32);                   // tokens per warp (>= 4)
+    constexpr int D = VPL <= 4 ? 4 : (VPL <= 8 ? 2 : 1);  // tokens in flight per warp
+    static_assert(32 / (warp_topk_threads<VPL>() / 32) % D == 0, "token groups");
+    constexpr int kMaxPerWarp = kMaxChunk / (kT / 32);
     __shared__ int s_hist[kMaxExperts];
+    // per warp, per token of the warp: the k selected keys' values and experts
+    // (written in the selection rounds, read back one token per lane; rows of
+    // kp = k | 1 words, so the lanes' reads fall in distinct banks)
+    __shared__ float s_z[kT / 32][kMaxPerWarp * (kMaxTopK + 1)];
+    __shared__ int32_t s_id[kT / 32][kMaxPerWarp * (kMaxTopK + 1)];
+    const int kp = k | 1;
     pdl_wait();
     pdl_trigger();
     for (int e = threadIdx.x; e < E; e += kT) s_hist[e] = 0;
@@ -191,7 +239,7 @@ route_topk_warp_kernel(const float* __restrict__ logits, const float* __restrict
     }
     __syncthreads();
 
-    const int t_warp = blockIdx.x * kChunk + warp * kPerWarp;
+    const int t_warp = blockIdx.x * ch + warp * per_warp;
     float cur[D][VPL], nxt[D][VPL];
 #pragma unroll
     for (int u = 0; u < D; ++u) {
@@ -199,8 +247,8 @@ route_topk_warp_kernel(const float* __restrict__ logits, const float* __restrict
         if (t < T) load_lane<VPL, VW>(logits + (size_t)t * E, lane_vw, E, cur[u]);
     }
 #pragma unroll 1
-    for (int g = 0; g < kPerWarp / D; ++g) {
-        if (g + 1 < kPerWarp / D) {
+    for (int g = 0; g < per_warp / D; ++g) {
+        if (g + 1 < per_warp / D) {
 #pragma unroll
             for (int u = 0; u < D; ++u) {
                 const int t = t_warp + (g + 1) * D + u;
@@ -212,52 +260,88 @@ route_topk_warp_kernel(const float* __restrict__ logits, const float* __restrict
             const int t = t_warp + g * D + u;
             if (t < T) {  // warp-uniform
                 uint32_t key[VPL];
+                int ex_i[VPL];  // expert of each slot
 #pragma unroll
                 for (int i = 0; i < VPL; ++i) {
                     const int e = (i / VW) * 32 * VW + lane_vw + i % VW;
+                    ex_i[i] = e;
                     key[i] = (e < E) ? route_key(__fadd_rn(cur[u][i], b[i])) : 0u;
                 }
-                float my_z = 0.0f;
-                int my_e = 0;
-                for (int r = 0; r < k; ++r) {
-                    uint32_t bk = 0u;
-                    int bi = INT_MAX;
+                const int tw = g * D + u;  // token index within the warp
+                float* zrow = s_z[warp] + tw * kp;
+                int32_t* idrow = s_id[warp] + tw * kp;
+                if constexpr (VPL <= 8) {
+                    // the lane's candidates sorted once, (key desc, expert asc); a
+                    // round takes the best head of the warp and its owner pops it
+                    sort_desc<VPL>(key, ex_i);
+                    for (int r = 0; r < k; ++r) {
+                        // k <= E, so some lane still holds an untaken expert: m > 0
+                        const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
+                        const int win = (int)__reduce_min_sync(
+                            0xffffffffu, key[0] == m ? (uint32_t)ex_i[0] : 0xffffffffu);
+                        if (ex_i[0] == win) {
 #pragma unroll
-                    for (int i = 0; i < VPL; ++i)
-                        if (key[i] > bk) {
-                            bk = key[i];
-                            bi = (i / VW) * 32 * VW + lane_vw + i % VW;
+                            for (int i = 0; i + 1 < VPL; ++i) {
+                                key[i] = key[i + 1];
+                                ex_i[i] = ex_i[i + 1];
+                            }
+                            key[VPL - 1] = 0u;
+                            ex_i[VPL - 1] = INT_MAX;
                         }
-                    // k <= E, so some lane still holds an untaken expert: m > 0
-                    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
-                    const int win = (int)__reduce_min_sync(
-                        0xffffffffu, bk == m ? (uint32_t)bi : 0xffffffffu);
-                    const int off = win - lane_vw;  // slot of the winner in its lane
-#pragma unroll
-                    for (int i = 0; i < VPL; ++i)
-                        if (off == (i / VW) * 32 * VW + i % VW) key[i] = 0u;
-                    if (lane == r) {
-                        my_z = key_value(m);
-                        my_e = win;
+                        if (lane == 0) {
+                            zrow[r] = key_value(m);
+                            idrow[r] = win;
+                        }
                     }
-                }
-                const float z0 = __shfl_sync(0xffffffffu, my_z, 0);
-                const float ex = (lane < k) ? expf(__fsub_rn(my_z, z0)) : 0.0f;
-                float s = 0.0f;
-                for (int i = 0; i < k; ++i) s = __fadd_rn(s, __shfl_sync(0xffffffffu, ex, i));
-                if (lane < k) {
-                    ids[(size_t)t * k + lane] = my_e;
-                    w[(size_t)t * k + lane] = __fdiv_rn(ex, s);
-                    if ((unsigned)my_e < (unsigned)E) atomicAdd(&s_hist[my_e], 1);
-                    else flag_error(err, MOE_DEVERR_EXPERT_INDEX);
+                } else {
+                    for (int r = 0; r < k; ++r) {
+                        uint32_t bk = 0u;
+                        int bi = INT_MAX;
+#pragma unroll
+                        for (int i = 0; i < VPL; ++i)
+                            if (key[i] > bk) {
+                                bk = key[i];
+                                bi = ex_i[i];
+                            }
+                        const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+                        const int win = (int)__reduce_min_sync(
+                            0xffffffffu, bk == m ? (uint32_t)bi : 0xffffffffu);
+#pragma unroll
+                        for (int i = 0; i < VPL; ++i)
+                            if (ex_i[i] == win) key[i] = 0u;
+                        if (lane == 0) {
+                            zrow[r] = key_value(m);
+                            idrow[r] = win;
+                        }
+                    }
                 }
             }
         }
-        if (g + 1 < kPerWarp / D) {
+        if (g + 1 < per_warp / D) {
 #pragma unroll
             for (int u = 0; u < D; ++u)
 #pragma unroll
                 for (int i = 0; i < VPL; ++i) cur[u][i] = nxt[u][i];
+        }
+    }
+    __syncwarp();
+    // lane j finishes the warp's token j: w_j = exp(z_j - z_0) / sum_i exp(z_i - z_0)
+    // (sum in rank order), the k ids and weights stored contiguously
+    {
+        const int t = t_warp + lane;
+        if (lane < per_warp && t < T) {
+            const float* zrow = s_z[warp] + lane * kp;
+            const int32_t* idrow = s_id[warp] + lane * kp;
+            const float z0 = zrow[0];
+            float sum = 0.0f;
+            for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, expf(__fsub_rn(zrow[j], z0)));
+            for (int j = 0; j < k; ++j) {
+                const int e = idrow[j];
+                ids[(size_t)t * k + j] = e;
+                w[(size_t)t * k + j] = __fdiv_rn(expf(__fsub_rn(zrow[j], z0)), sum);
+                if ((unsigned)e < (unsigned)E) atomicAdd(&s_hist[e], 1);
+                else flag_error(err, MOE_DEVERR_EXPERT_INDEX);
+            }
         }
     }
     __syncthreads();
@@ -313,22 +397,23 @@ route_scan_kernel(const int32_t* __restrict__ chunk_hist, int nchunks, int E, in
 }
 
 // ------------------------------------------------------------------- K3 ----
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kMaxChunk)
 route_assign_kernel(const int32_t* __restrict__ ids, int T, int E, int k, int capacity,
-                    int nchunks, const int32_t* __restrict__ chunk_base,
+                    int ch, int nchunks, const int32_t* __restrict__ chunk_base,
                     const int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
                     int32_t* __restrict__ n_dropped, int32_t* __restrict__ slot_row,
                     int32_t* __restrict__ row_slot, int32_t* err) {
-    __shared__ uint32_t s_mask[kWarps][kMaxExperts];
+    __shared__ uint32_t s_mask[kMaxWarps][kMaxExperts];
     __shared__ int32_t s_base[kMaxExperts];
     __shared__ int32_t s_off[kMaxExperts + 1];
-    __shared__ int32_t s_warp[kWarps];
+    __shared__ int32_t s_warp[kMaxWarps];
     pdl_wait();
     pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nthr = blockDim.x, nwarps = nthr >> 5;  // blockDim.x == ch
 
     // offsets: exclusive scan of kept over the experts, per = experts a thread holds
-    const int per = (E + kThreads - 1) / kThreads;
+    const int per = (E + nthr - 1) / nthr;
     const int e0 = tid * per;
     int32_t loc = 0;
     for (int i = 0; i < per; ++i)
@@ -340,16 +425,15 @@ route_assign_kernel(const int32_t* __restrict__ ids, int T, int E, int k, int ca
         if (lane >= off) incl += o;
     }
     if (lane == 31) s_warp[warp] = incl;
-    for (int e = tid; e < E; e += kThreads) {
+    for (int e = tid; e < E; e += nthr) {
         s_base[e] = blockIdx.x < nchunks ? chunk_base[(size_t)blockIdx.x * E + e] : 0;
 #pragma unroll
-        for (int wv = 0; wv < kWarps; ++wv) s_mask[wv][e] = 0u;
+        for (int wv = 0; wv < kMaxWarps; ++wv) s_mask[wv][e] = 0u;
     }
     __syncthreads();
     int32_t run = incl - loc;
     int32_t total = 0;
-#pragma unroll
-    for (int wv = 0; wv < kWarps; ++wv) {
+    for (int wv = 0; wv < nwarps; ++wv) {
         if (wv < warp) run += s_warp[wv];
         total += s_warp[wv];
     }
@@ -361,11 +445,11 @@ route_assign_kernel(const int32_t* __restrict__ ids, int T, int E, int k, int ca
     if (tid == 0) s_off[E] = total;
     __syncthreads();
     if (blockIdx.x == 0) {
-        for (int e = tid; e <= E; e += kThreads) offsets[e] = s_off[e];
+        for (int e = tid; e <= E; e += nthr) offsets[e] = s_off[e];
         if (tid == 0) n_dropped[0] = (int32_t)((int64_t)T * k - total);
     }
 
-    const int t = blockIdx.x * kChunk + tid;
+    const int t = blockIdx.x * ch + tid;
     const bool active = t < T;
     const int32_t* my_ids = ids + (size_t)t * k;
     if (active)
@@ -401,66 +485,71 @@ route_assign_kernel(const int32_t* __restrict__ ids, int T, int E, int k, int ca
 static size_t align256(size_t v) { return (v + 255u) & ~size_t(255u); }
 
 template <int EMAX, int KMAX>
-static int launch_lane(int nchunks, cudaStream_t st, const float* logits, const float* bias,
-                       int T, int E, int k, int vw, int32_t* ids, float* w, int32_t* hist) {
-    return launch_pdl(route_topk_lane_kernel<EMAX, KMAX>, nchunks, kThreads, 0, st, logits, bias,
-                      T, E, k, vw, ids, w, hist, device_error_word());
+static int launch_lane(int nchunks, int ch, cudaStream_t st, const float* logits,
+                       const float* bias, int T, int E, int k, int vw, int32_t* ids, float* w,
+                       int32_t* hist) {
+    return launch_pdl(route_topk_lane_kernel<EMAX, KMAX>, nchunks, ch, 0, st, logits, bias, T, E,
+                      k, vw, ch, ids, w, hist, device_error_word());
 }
 template <int EMAX>
-static int launch_lane_k(int nchunks, cudaStream_t st, const float* logits, const float* bias,
-                         int T, int E, int k, int vw, int32_t* ids, float* w, int32_t* hist) {
-    if (k <= 2) return launch_lane<EMAX, 2>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
-    if (k <= 8) return launch_lane<EMAX, 8>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
-    return launch_lane<EMAX, EMAX>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
+static int launch_lane_k(int nchunks, int ch, cudaStream_t st, const float* logits,
+                         const float* bias, int T, int E, int k, int vw, int32_t* ids, float* w,
+                         int32_t* hist) {
+    if (k <= 2)
+        return launch_lane<EMAX, 2>(nchunks, ch, st, logits, bias, T, E, k, vw, ids, w, hist);
+    if (k <= 8)
+        return launch_lane<EMAX, 8>(nchunks, ch, st, logits, bias, T, E, k, vw, ids, w, hist);
+    return launch_lane<EMAX, EMAX>(nchunks, ch, st, logits, bias, T, E, k, vw, ids, w, hist);
 }
 template <int VPL>
-static int launch_warp(int nchunks, cudaStream_t st, const float* logits, const float* bias,
-                       int T, int E, int k, bool vec, int32_t* ids, float* w, int32_t* hist) {
+static int launch_warp(int nchunks, int ch, cudaStream_t st, const float* logits,
+                       const float* bias, int T, int E, int k, bool vec, int32_t* ids, float* w,
+                       int32_t* hist) {
     constexpr int VW = VPL >= 4 ? 4 : VPL;
     if (vec)
         return launch_pdl(route_topk_warp_kernel<VPL, VW>, nchunks, warp_topk_threads<VPL>(), 0,
-                          st, logits, bias, T, E, k, ids, w, hist, device_error_word());
+                          st, logits, bias, T, E, k, ch, ids, w, hist, device_error_word());
     return launch_pdl(route_topk_warp_kernel<VPL, 1>, nchunks, warp_topk_threads<VPL>(), 0, st,
-                      logits, bias, T, E, k, ids, w, hist, device_error_word());
+                      logits, bias, T, E, k, ch, ids, w, hist, device_error_word());
 }
 
-// The three launches of one routing call; `scratch` is 256-byte aligned and
-// holds at least route_scratch_bytes(T, E).
-static size_t route_scratch_bytes(int T, int E) {
-    const size_t nchunks = ((size_t)T + kChunk - 1) / kChunk;
+// The three launches of one routing call in chunks of ch tokens; `scratch` is
+// 256-byte aligned and holds at least route_scratch_bytes(T, E, ch).
+static size_t route_scratch_bytes(int T, int E, int ch) {
+    const size_t nchunks = ((size_t)T + ch - 1) / ch;
     return 2 * align256(nchunks * (size_t)E * sizeof(int32_t));
 }
 
 static int launch_route(const float* logits, const float* bias, int T, int E, int k, int capacity,
                         int32_t* ids, float* w, int32_t* counts, int32_t* kept, int32_t* offsets,
                         int32_t* slot_row, int32_t* row_slot, int32_t* n_dropped, char* scratch,
-                        cudaStream_t st) {
-    const int nchunks = (T + kChunk - 1) / kChunk;
+                        int ch, cudaStream_t st) {
+    const int nchunks = (T + ch - 1) / ch;
     int32_t* hist = reinterpret_cast<int32_t*>(scratch);
     int32_t* base = reinterpret_cast<int32_t*>(scratch + align256((size_t)nchunks * E * 4));
     if (T > 0) {
         // widest load the row layout and the pointer's alignment allow
         const uintptr_t p = reinterpret_cast<uintptr_t>(logits);
         const int vw = (E % 4 == 0 && p % 16 == 0) ? 4 : (E % 2 == 0 && p % 8 == 0) ? 2 : 1;
+        const int n = nchunks;
         int rc;
-        if (E <= 8) rc = launch_lane_k<8>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
-        else if (E <= 16) rc = launch_lane_k<16>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
-        else if (E <= 32) rc = launch_lane_k<32>(nchunks, st, logits, bias, T, E, k, vw, ids, w, hist);
-        else if (E <= 64) rc = launch_warp<2>(nchunks, st, logits, bias, T, E, k, vw >= 2, ids, w, hist);
-        else if (E <= 128) rc = launch_warp<4>(nchunks, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
-        else if (E <= 256) rc = launch_warp<8>(nchunks, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
-        else if (E <= 512) rc = launch_warp<16>(nchunks, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
-        else rc = launch_warp<32>(nchunks, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
+        if (E <= 8) rc = launch_lane_k<8>(n, ch, st, logits, bias, T, E, k, vw, ids, w, hist);
+        else if (E <= 16) rc = launch_lane_k<16>(n, ch, st, logits, bias, T, E, k, vw, ids, w, hist);
+        else if (E <= 32) rc = launch_lane_k<32>(n, ch, st, logits, bias, T, E, k, vw, ids, w, hist);
+        else if (E <= 64) rc = launch_warp<2>(n, ch, st, logits, bias, T, E, k, vw >= 2, ids, w, hist);
+        else if (E <= 128) rc = launch_warp<4>(n, ch, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
+        else if (E <= 256) rc = launch_warp<8>(n, ch, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
+        else if (E <= 512) rc = launch_warp<16>(n, ch, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
+        else rc = launch_warp<32>(n, ch, st, logits, bias, T, E, k, vw == 4, ids, w, hist);
         if (rc != MOE_OK) return MOE_ERR_CUDA;
     }
     if (launch_pdl(route_scan_kernel, (E + 31) / 32, kScanThreads, 0, st, (const int32_t*)hist,
                    nchunks, E, capacity, base, counts, kept) != MOE_OK)
         return MOE_ERR_CUDA;
     // at least one CTA: it writes offsets and n_dropped even when T = 0
-    if (launch_pdl(route_assign_kernel, nchunks > 0 ? nchunks : 1, kThreads, 0, st,
-                   (const int32_t*)ids, T, E, k, capacity, nchunks, (const int32_t*)base,
-                   (const int32_t*)kept, offsets, n_dropped, slot_row, row_slot,
-                   device_error_word()) != MOE_OK)
+    if (launch_pdl(route_assign_kernel, nchunks > 0 ? nchunks : 1, ch, 0, st, (const int32_t*)ids,
+                   T, E, k, capacity, ch, nchunks, (const int32_t*)base, (const int32_t*)kept,
+                   offsets, n_dropped, slot_row, row_slot, device_error_word()) != MOE_OK)
         return MOE_ERR_CUDA;
     return MOE_OK;
 }
@@ -483,7 +572,7 @@ using namespace moe;
 extern "C" MOE_API size_t moe_route_workspace_size(int T, int E, int k) {
     (void)k;
     if (T < 0 || E <= 0) return 0;
-    return route_scratch_bytes(T, E) + 256;  // + slack to align the caller's pointer
+    return route_scratch_bytes(T, E, chunk_tokens(T)) + 256;  // + slack to align the pointer
 }
 
 extern "C" MOE_API int moe_route(const float* logits, const float* bias, int T, int E, int k, int capacity,
@@ -498,7 +587,8 @@ extern "C" MOE_API int moe_route(const float* logits, const float* bias, int T, 
     char* ws = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(workspace) + 255u) &
                                        ~uintptr_t(255u));
     return launch_route(logits, bias, T, E, k, capacity, ids, w, counts, kept, offsets, slot_row,
-                        row_slot, n_dropped, ws, reinterpret_cast<cudaStream_t>(stream));
+                        row_slot, n_dropped, ws, chunk_tokens(T),
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------------------
@@ -547,11 +637,11 @@ extern "C" MOE_API int moe_route_noalloc(const float* logits, const float* bias,
     const int rc = check_route_args(logits, T, E, k, ids, w, counts, kept, offsets, slot_row,
                                     row_slot, n_dropped);
     if (rc != MOE_OK) return rc;
-    // The fixed scratch bounds the problem size.
-    if (moe_route_workspace_size(T, E, k) > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
+    // The fixed scratch bounds the problem size (128-token chunks whatever T).
+    if (route_scratch_bytes(T, E, kMaxChunk) + 256 > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
     void* scratch = noalloc_scratch_ptr();
     if (!scratch) return MOE_ERR_CUDA;
     return launch_route(logits, bias, T, E, k, capacity, ids, w, counts, kept, offsets, slot_row,
-                        row_slot, n_dropped, static_cast<char*>(scratch),
+                        row_slot, n_dropped, static_cast<char*>(scratch), kMaxChunk,
                         reinterpret_cast<cudaStream_t>(stream));
 }
