@@ -70,7 +70,7 @@ extern "C" MOE_API int moe_gate(const void* x, const void* Wg, int dtype, int T,
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // fp32 layers with few experts: the CUDA-core kernel (measured faster than
     // the tiled SIMT GEMM there); bf16 stays on the tensor cores, which were
-    // measured faster than that kernel.
+    // measured faster than that kernel (skewed_drops: 15.0 vs 16.2 us).
     if (dtype == MOE_DTYPE_F32 && gate_small_fits(E, d, dtype))
         return launch_gate_small(x, Wg, dtype, T, d, E, logits, st);
     if (dtype == MOE_DTYPE_BF16)

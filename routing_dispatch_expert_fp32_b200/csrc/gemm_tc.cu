@@ -48,9 +48,10 @@ constexpr long long kPairMinRowsPerGroup = MOE_PAIR_MIN_ROWS_PER_GROUP;
 // Dense groups: pair tiles for whole 256-row blocks plus 1-CTA tiles for the
 // tails (0: pair tiles for everything).
 #ifndef MOE_SPLIT_TAILS
-#define MOE_SPLIT_TAILS 0
+#define MOE_SPLIT_TAILS 1
 #endif
 constexpr bool kSplitTails = MOE_SPLIT_TAILS != 0;
+
 
 template <int BN>
 struct Cfg {

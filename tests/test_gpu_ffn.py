@@ -88,6 +88,29 @@ def test_ffn_dense_groups_elementwise(moe, sizes, d, F):
     assert moe.moe_device_error() == 0
 
 
+@pytest.mark.parametrize("sizes,d,F", [
+    ([1, 15, 16, 17, 63, 64, 65, 0, 127, 128, 129, 255, 256, 257, 3], 128, 256),
+    ([40, 0, 129, 7, 300, 2, 16], 200, 512),          # K tail in the first GEMM
+    ([5, 130, 61, 1, 0, 250], 512, 768),
+])
+def test_ffn_sparse_groups_with_many_tiles_elementwise(moe, sizes, d, F):
+    """A row capacity of three or more waves of 128-row tiles (the sparse
+    regime of the large workloads): 1-CTA tiles, many per CTA."""
+    E = len(sizes)
+    R = sum(sizes)
+    offsets = np.array([0] + np.cumsum(sizes).tolist(), np.int32)
+    Xp = rand((R, d), 1.0, "bf16", 21)
+    W1 = rand((E, F, d), d ** -0.5, "bf16", 22)
+    W2 = rand((E, d, F), F ** -0.5, "bf16", 23)
+    Rmax = 60000
+    H, Yp = run_ffn(moe, Xp, W1, W2, offsets, Rmax)
+    Yr, Hr = oracle.expert_ffn(Xp, W1, W2, offsets, want_h=True)
+    assert_close(H[:R], Hr, "H")
+    assert_close(Yp[:R], Yr, "Yp")
+    assert not H[R:].any() and not Yp[R:].any()
+    assert moe.moe_device_error() == 0
+
+
 def test_ffn_relu_kills_negative_first_layer(moe):
     E, d, F = 2, 128, 256
     Xp = wl.to_bf16_bits(np.abs(np.random.default_rng(0).standard_normal((300, d))) + 0.1)

@@ -46,8 +46,9 @@ def _rand(shape, scale, seed):
     return wl.to_bf16_bits(a)
 
 
-# (sizes, d, F, R_max) reaching each forward kernel in both GEMMs:
-#   pair, pair_wide  R_max >= 1024 rows per expert: 2-CTA 256 x 256 tiles;
+# (sizes, d, F, R_max) reaching each forward kernel:
+#   pair, pair_wide  R_max >= 1024 rows per expert: 2-CTA 256 x 256 tiles for
+#                    whole 256-row blocks, 1-CTA 128 x 256 tiles for the tails;
 #   one_cta, ragged  sparse groups with at least three waves of 128-row tiles:
 #                    1-CTA 128 x 256 tiles (ragged adds groups of several tiles)
 _SMALL = [int(v) for v in np.random.default_rng(7).integers(0, 41, 64)]
