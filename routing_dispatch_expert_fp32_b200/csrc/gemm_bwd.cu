@@ -45,11 +45,22 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 512;
 constexpr int MN_BOX = 64;                    // MN elements per box (128 bytes)
 constexpr int MN_BOX_BYTES = MN_BOX * BK * 2;  // 8 KB
+// Epilogue warps: two per TMEM lane quadrant, each draining half of the 256
+// accumulator columns (4: one per quadrant, all columns).  The weight-gradient
+// tiles have short K loops, so a tile's time is mostly its epilogue.
+#ifndef MOE_BWD_EPI_WARPS
+#define MOE_BWD_EPI_WARPS 8
+#endif
+constexpr int kEpiWarps = MOE_BWD_EPI_WARPS;
+static_assert(kEpiWarps == 4 || kEpiWarps == 8, "epilogue warps");
+constexpr int kBwdThreads = 64 + 32 * kEpiWarps;  // TMA warp, MMA warp, epilogue
+constexpr int kBwdEpiThreads = 32 * kEpiWarps;
+constexpr int kColsPerWarp = BN / (kEpiWarps / 4);
 // fp32 epilogue: per warp kEpiBufs staging tiles of 32 rows x 32 columns,
 // written in turn while earlier tensor stores drain; the operand ring gives
-// up one stage for them (the weight-gradient tiles have short K loops).
-constexpr int kEpiBufs = 4;
-constexpr int EPI_STAGE_BYTES = 4 * kEpiBufs * 32 * 128;
+// up one stage for them (64 KB in all).
+constexpr int kEpiBufs = kEpiWarps == 8 ? 2 : 4;
+constexpr int EPI_STAGE_BYTES = kEpiWarps * kEpiBufs * 32 * 128;
 constexpr int stages_for(int EPI) { return EPI == 2 ? 3 : kStages; }
 template <int EPI>
 constexpr int fixed_bytes() {
@@ -90,7 +101,7 @@ __device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
 __device__ __forceinline__ float bf(uint32_t u, int hi) { return hi ? bf16hi(u) : bf16lo(u); }
 
 template <bool A_MN, bool KVAR, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
 gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
                 const __grid_constant__ CUtensorMap tmap_c, const BwdArgs args, int32_t* err) {
@@ -127,7 +138,7 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull + a, 1);
-            mbar_init(tempty + a, kEpiThreads);
+            mbar_init(tempty + a, kBwdEpiThreads);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -147,7 +158,7 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
         mt_fix = (M_fix + BM - 1) / BM;
         total = E * mt_fix * nt;
         // the group bounds every role reads per tile, kept in shared memory
-        for (int i = threadIdx.x; i <= E; i += kThreads)
+        for (int i = threadIdx.x; i <= E; i += kBwdThreads)
             s_prefix[i] = offsets ? offsets[i] : min(single_M, i * slice_rows);
         if (offsets && threadIdx.x == 0) {  // validate the offsets the K loops will follow
             for (int e = 0; e < E; ++e) {
@@ -327,28 +338,32 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
         __syncwarp();
     } else {
         // ---------------------------------------------------- epilogue
+        // warp 2 + ew drains TMEM lane quadrant warp % 4 (a warp's fixed
+        // quadrant), columns [c_lo, c_lo + kColsPerWarp) of the accumulator
+        const int ew = warp - 2;
         const int quad = warp & 3;
+        const int c_lo = (ew >> 2) * kColsPerWarp;
         const int row = quad * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-        uint8_t* stage_c = sC + quad * (kEpiBufs * 4096);  // this warp's staging tiles
+        uint8_t* stage_c = sC + ew * (kEpiBufs * 4096);  // this warp's staging tiles
         int it = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
             int e, m0, rows, n0, k0, nk, kr;
             coord(tile, e, m0, rows, n0, k0, nk, kr);
             const int acc = it & 1;
             const bool row_ok = row < rows;
-            // dH: the ReLU mask of this row's 256 columns, as bits, loaded from
-            // H while the tile's MMAs still run (bit i of word w: column
-            // n0 + 32 w + i has H > 0)
-            uint32_t hm[BN / 32];
+            // dH: the ReLU mask of this row's columns, as bits, loaded from H
+            // while the tile's MMAs still run (bit i of word w: column
+            // n0 + c_lo + 32 w + i has H > 0)
+            uint32_t hm[kColsPerWarp / 32];
 #pragma unroll
-            for (int w = 0; w < BN / 32; ++w) hm[w] = 0u;
+            for (int w = 0; w < kColsPerWarp / 32; ++w) hm[w] = 0u;
             if (EPI == EPI_BF16_RELU_MASK && row_ok) {
-                const uint4* h =
-                    reinterpret_cast<const uint4*>(Hmask + static_cast<size_t>(m0 + row) * N + n0);
-                const int nv = min(BN, N - n0) / 8;
+                const uint4* h = reinterpret_cast<const uint4*>(
+                    Hmask + static_cast<size_t>(m0 + row) * N + n0 + c_lo);
+                const int nv = min(kColsPerWarp, N - n0 - c_lo) / 8;
 #pragma unroll
-                for (int b = 0; b < BN / 64; ++b) {
+                for (int b = 0; b < kColsPerWarp / 64; ++b) {
                     uint4 v[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
@@ -373,7 +388,7 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 // rows past M_fix and columns past N are clipped by the map
                 const bool rows_in = m0 + quad * 32 < M_fix;
 #pragma unroll 1
-                for (int cb = 0; cb < BN; cb += 32 * kEpiBufs) {
+                for (int cb = c_lo; cb < c_lo + kColsPerWarp; cb += 32 * kEpiBufs) {
                     if (lane == 0) bulk_wait_read_allow<0>();  // the last batch has been read
                     __syncwarp();
 #pragma unroll
@@ -403,13 +418,13 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
             } else {
 #pragma unroll 1
-                for (int cc = 0; cc < BN; cc += 32) {
+                for (int cc = c_lo; cc < c_lo + kColsPerWarp; cc += 32) {
                     uint32_t r[32];
                     tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + cc), r);
                     const int col = n0 + cc;
                     const uint32_t mw = hm[0];
 #pragma unroll
-                    for (int w = 0; w + 1 < BN / 32; ++w) hm[w] = hm[w + 1];
+                    for (int w = 0; w + 1 < kColsPerWarp / 32; ++w) hm[w] = hm[w + 1];
                     if (!row_ok || col >= N) continue;
                     __nv_bfloat16* dst =
                         static_cast<__nv_bfloat16*>(Cv) + static_cast<size_t>(m0 + row) * N + col;
@@ -457,7 +472,7 @@ int launch_bwd(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
     if (ensure_smem<gemm_bwd_kernel<A_MN, KVAR, EPI>>(smem) != MOE_OK) return MOE_ERR_CUDA;
     const int grid = test_cap((int)(ub < num_sms() ? ub : num_sms()));
     if (grid <= 0) return MOE_OK;
-    return launch_pdl(gemm_bwd_kernel<A_MN, KVAR, EPI>, grid, kThreads, smem, st, ta, tb, tc_map,
+    return launch_pdl(gemm_bwd_kernel<A_MN, KVAR, EPI>, grid, kBwdThreads, smem, st, ta, tb, tc_map,
                       args, device_error_word());
 }
 
