@@ -9,6 +9,8 @@ time through the runtime's driver entry points).
 from __future__ import annotations
 
 import concurrent.futures
+import contextlib
+import fcntl
 import glob
 import os
 import subprocess
@@ -51,11 +53,27 @@ def _compile(src: str, verbose: bool, extra, build_dir) -> str:
     return obj
 
 
+@contextlib.contextmanager
+def _lock():
+    """One build at a time (test workers may start builds concurrently)."""
+    os.makedirs(BUILD, exist_ok=True)
+    with open(os.path.join(BUILD, ".lock"), "w") as f:
+        fcntl.flock(f, fcntl.LOCK_EX)
+        try:
+            yield
+        finally:
+            fcntl.flock(f, fcntl.LOCK_UN)
+
+
 def build(force: bool = False, verbose: bool = False, extra=(), out: str = LIB) -> str:
     """Builds `out` (default: the package's libmoe.so); `extra` are added nvcc
     flags (e.g. -D tuning constants) and force a rebuild into a separate
     object directory."""
-    extra = list(extra)
+    with _lock():
+        return _build(force, verbose, list(extra), out)
+
+
+def _build(force, verbose, extra, out):
     if not force and not extra and out == LIB and up_to_date():
         return LIB
     build_dir = BUILD if not extra else os.path.join(BUILD, "variant_" + "_".join(
