@@ -382,37 +382,35 @@ gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmap_a,
             if (!mbar_wait(tfull + acc, (it >> 1) & 1, abort_flag, err)) break;
             tc_fence_after();
             if (EPI == EPI_F32) {
-                // fp32 weight gradient: kEpiBufs 32 x 32 blocks of the warp's
-                // rows at a time are staged in shared memory (128-byte swizzle)
-                // behind one proxy fence, then written by one tensor store each;
+                // fp32 weight gradient: the warp's 32 x 32 blocks go one at a time
+                // through its kEpiBufs staging buffers (128-byte swizzle), each
+                // written by one tensor store while the next block is staged;
                 // rows past M_fix and columns past N are clipped by the map
                 const bool rows_in = m0 + quad * 32 < M_fix;
 #pragma unroll 1
-                for (int cb = c_lo; cb < c_lo + kColsPerWarp; cb += 32 * kEpiBufs) {
-                    if (lane == 0) bulk_wait_read_allow<0>();  // the last batch has been read
+                for (int cb = c_lo; cb < c_lo + kColsPerWarp; cb += 32) {
+                    // one 32 x 32 block per step into staging buffer (step % kEpiBufs);
+                    // the store that last used that buffer was committed kEpiBufs
+                    // groups ago, so wait until at most kEpiBufs - 1 groups still read
+                    const int u = ((cb - c_lo) >> 5) % kEpiBufs;
+                    if (lane == 0) bulk_wait_read_allow<kEpiBufs - 1>();
                     __syncwarp();
+                    uint32_t r[32];
+                    tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + cb), r);
+                    if (nk == 0) {
 #pragma unroll
-                    for (int u = 0; u < kEpiBufs; ++u) {
-                        uint32_t r[32];
-                        tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + cb + 32 * u),
-                                  r);
-                        if (nk == 0) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) r[i] = 0u;  // group without rows
-                        }
-                        uint8_t* buf = stage_c + u * 4096;
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            *reinterpret_cast<uint4*>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
-                                make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+                        for (int i = 0; i < 32; ++i) r[i] = 0u;  // group without rows
                     }
+                    uint8_t* buf = stage_c + u * 4096;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<uint4*>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                            make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
-                    if (lane == 0 && rows_in) {
-                        for (int u = 0; u < kEpiBufs; ++u) {
-                            const int col = n0 + cb + 32 * u;
-                            if (col < N) tma_store_3d(&tmap_c, stage_c + u * 4096, col, m0 + quad * 32, e);
-                        }
+                    if (lane == 0) {
+                        const int col = n0 + cb;
+                        if (rows_in && col < N) tma_store_3d(&tmap_c, buf, col, m0 + quad * 32, e);
                         bulk_commit();
                     }
                 }

@@ -103,7 +103,8 @@ __device__ inline int build_tile_table(const int32_t* __restrict__ offsets, int 
 
 // Maps a linear tile index to its coordinates, given the prefix of M-tiles per
 // group (s_prefix from build_tile_table with nt = 1 and the same part) and nt
-// N-tiles per group: group e owns tiles [nt * s_prefix[e], nt * s_prefix[e+1]).
+// N-tiles per group: group e owns tiles [nt * s_prefix[e], nt * s_prefix[e+1]),
+// its M-tiles fastest.
 __device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* s_prefix, int E,
                                                 const int32_t* __restrict__ offsets, int single_M,
                                                 int BM, int BN, int nt, int part = PART_ALL) {
@@ -113,11 +114,11 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* s_prefi
         if (nt * s_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
     }
     const int e = lo;
-    int a, m;
-    group_part(offsets, e, single_M, part, a, m);
-    const int mt = (m + BM - 1) / BM;
+    const int mt = s_prefix[e + 1] - s_prefix[e];
     const int local = tile - nt * s_prefix[e];
     const int mb = local % mt, nb = local / mt;
+    int a, m;
+    group_part(offsets, e, single_M, part, a, m);
     TileCoord c;
     c.e = e;
     c.row0 = a + mb * BM;
