@@ -180,3 +180,36 @@ def test_route_unaligned_logits_take_the_scalar_loads(moe, E):
     for name in ["ids", "counts", "offsets", "slot_row"]:
         assert np.array_equal(host(out[name]), r[name]), name
     np.testing.assert_allclose(host(out["w"]), r["w"], rtol=4e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("T,E,k,cap", [
+    (1000, 36, 3, 0), (999, 68, 1, 40), (4100, 100, 8, 0), (333, 132, 5, 9), (2049, 252, 6, 0),
+    (40000, 64, 2, 700), (20000, 200, 7, 0), (1, 64, 8, 0), (31, 128, 4, 1),
+])
+def test_route_tiled_shapes(moe, T, E, k, cap):
+    """Shapes of the TMA-tiled kernel (32 < E <= 256, E % 4 == 0, k <= 8): partial
+    last slabs, skipped slabs, every chunk size (32, 64, 128 tokens) and
+    ragged last chunks."""
+    rng = np.random.default_rng(T + 3 * E + k)
+    logits = rng.standard_normal((T, E), dtype=np.float32)
+    bias = (0.5 * rng.standard_normal(E)).astype(np.float32)
+    check_route(moe, logits, bias, k, cap)
+
+
+@pytest.mark.parametrize("E,k", [(64, 2), (96, 5), (128, 4), (256, 8)])
+def test_route_near_and_exact_ties_for_many_experts(moe, E, k):
+    """Scores a few units in the last place apart, and exact integer ties, so
+    that the selection's truncated keys collide and tokens are ranked again
+    exactly; -0.0 logits and a -0.0 bias tie with +0.0."""
+    rng = np.random.default_rng(E + k)
+    T = 700
+    base = rng.standard_normal((T, 1)).astype(np.float32)
+    steps = rng.integers(-3, 4, (T, E)).astype(np.float32)
+    near = (base + steps * np.float32(1.2e-7) * np.abs(base)).astype(np.float32)
+    check_route(moe, near, None, k, 0)
+    ints = rng.integers(-2, 3, (T, E)).astype(np.float32)
+    ints[3] = 0.0
+    ints[4, ::2] = -0.0
+    bias = np.zeros(E, np.float32)
+    bias[::3] = -0.0
+    check_route(moe, ints, bias, k, 25)
