@@ -501,10 +501,12 @@ def measure(ctx: Ctx, w: wl.Workload, steps: int, warmup: int, full: bool):
         ev[5].record(stream)
 
     # R per batch (untimed): algorithmic work of each step
-    R_of = []
+    # and U, the tokens with at least one kept slot (input encode reads their rows)
+    R_of, U_of = [], []
     for i in range(nb):
         step(i)
         R_of.append(int(layer.offsets[-1].item()))
+        U_of.append(int((layer.slot_row >= 0).any(dim=1).sum().item()))
     # CUDA graphs per input batch: one graph of the whole step on one rank; with
     # several ranks two graphs (gate + route, the rest) around the NCCL
     # all_reduce of the counts.
@@ -651,13 +653,14 @@ def measure(ctx: Ctx, w: wl.Workload, steps: int, warmup: int, full: bool):
 
     # ---- per-stage numbers and the dominant kernel's roofline ----
     R_mean = float(np.mean([R_of[i % nb] for i in range(stage_steps)]))
+    U_mean = float(np.mean([U_of[i % nb] for i in range(stage_steps)]))
     names = ["gate", "route+popularity", "dispatch", "expert_ffn", "combine"]
     es = 2 if w.dtype == "bf16" else 4
     per = {}
     alg = {
         "gate": (2.0 * w.T * w.d * w.E, "flop") if not w.logits_direct else (0, "flop"),
         "route+popularity": (w.T * w.E * 4 + w.T * w.k * 4 * 4 + R_mean * 4, "byte"),
-        "dispatch": ((0 if layer.fused else w.T * w.d * es + R_mean * w.d * es
+        "dispatch": ((0 if layer.fused else U_mean * w.d * es + R_mean * w.d * es
                       + w.T * w.k * 4), "byte"),
         "expert_ffn": (4.0 * R_mean * w.d * w.F, "flop"),
         "combine": (R_mean * w.d * es + w.T * w.d * es + w.T * w.k * 8, "byte"),
@@ -677,6 +680,7 @@ def measure(ctx: Ctx, w: wl.Workload, steps: int, warmup: int, full: bool):
         per[n] = ent
     out["stages"] = per
     out["R_mean"] = R_mean
+    out["U_mean"] = U_mean
     if w.identity_experts:
         dom = "dispatch" if per["dispatch"]["ms"] >= per["combine"]["ms"] else "combine"
         amount = alg[dom][0]
