@@ -621,6 +621,11 @@ def measure(ctx: Ctx, w: wl.Workload, steps: int, warmup: int, full: bool):
         stage_ms += np.array([e[j].elapsed_time(e[j + 1]) for j in range(nev - 1)])
     stage_total_ms = float(stage_ms.sum())
     stage_ms /= stage_steps
+    # input encode and output decode alone (the layer holds the stage pass's last batch)
+    kernel_times = {}
+    if rank == 0 and w.dtype == "bf16":
+        kernel_times = permute_kernel_times(ctx, w, layer,
+                                            batches[(stage_steps - 1) % nb]["x"], peaks)
 
     out = {"elapsed_ms": elapsed_ms, "steps": steps,
            "value": w.T * steps * world / (elapsed_ms * 1e-3),
@@ -678,6 +683,8 @@ def measure(ctx: Ctx, w: wl.Workload, steps: int, warmup: int, full: bool):
                 ent["gbs"] = amount / (ms * 1e-3) / 1e9
                 ent["frac_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
         per[n] = ent
+    for name, v in kernel_times.items():
+        per[name]["kernel"] = v
     out["stages"] = per
     out["R_mean"] = R_mean
     out["U_mean"] = U_mean
@@ -857,6 +864,61 @@ def e2e_measure(ctx, w, steps, nb, batches, weights, layer, layers, conc, use_gr
     e2e_ms = ctx.max_over_ranks(e0.elapsed_time(e1))
     return {"e2e": {"value": w.T * e2e_steps * ctx.world / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "note": note}}
+
+
+def permute_kernel_times(ctx, w, layer, x, peaks, reps=8, n_rep=5):
+    """Input encode and output decode alone: back-to-back launches inside one CUDA
+    graph (programmatic launch, as in the step's graph), rotating over enough
+    copies of their buffers that a round moves more than twice the L2, so each
+    launch streams HBM.  The layer holds the routing of its last batch; the bytes
+    are that batch's (U tokens with a kept slot, R kept rows)."""
+    torch, moe = ctx.torch, ctx.moe
+    es = x.element_size()
+    R = int(layer.offsets[-1].item())
+    U = int((layer.slot_row >= 0).any(dim=1).sum().item())
+    l2 = getattr(torch.cuda.get_device_properties(ctx.local), "L2_cache_size", 126 << 20)
+    jobs = {}
+    if not layer.fused:
+        jobs["dispatch"] = U * w.d * es + R * w.d * es + w.T * w.k * 4
+    jobs["combine"] = R * w.d * es + w.T * w.d * es + w.T * w.k * 8
+    out = {}
+    wts = None if layer.fused else layer.w
+    for name, nbytes in jobs.items():
+        if nbytes <= 0:
+            continue
+        n_sets = int(min(16, max(2, -(-2 * l2 // nbytes))))
+        if name == "dispatch":
+            sets = [(x, layer.Xp)] + [(x.clone(), torch.empty_like(layer.Xp))
+                                      for _ in range(n_sets - 1)]
+            call = lambda a, b: moe.moe_dispatch(a, w.k, layer.slot_row, b)  # noqa: E731
+        else:
+            sets = [(layer.Yp, layer.y)] + [(layer.Yp.clone(), torch.empty_like(layer.y))
+                                            for _ in range(n_sets - 1)]
+            call = lambda a, b: moe.moe_combine(a, w.k, layer.slot_row, wts, b)  # noqa: E731
+        for a, b in sets:  # warm: loads the kernels, sets attributes outside the capture
+            call(a, b)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                for a, b in sets:
+                    call(a, b)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_rep):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / (n_rep * reps * n_sets)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"ms": ms, "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                     "bytes_per_launch": nbytes, "launches": n_rep * reps * n_sets,
+                     "buffer_sets": n_sets}
+        del g, sets
+        torch.cuda.empty_cache()
+    return out
 
 
 def f2_f4_backward_extras(ctx, w, step, nb, batches, weights, layer, stream):
