@@ -12,13 +12,14 @@
 // Both are HBM-bound row copies.  Token-parallel: one warp owns one token row
 // at a time (grid-stride over tokens), moves it in 16-byte vectors with
 // U vectors per lane in flight, and
-//   dispatch: reads x[t] once and writes it to each of its kept rows;
+//   dispatch: reads x[t] once and writes it to each of its kept rows (a token
+//             with no kept row is not read);
 //   combine:  reads the token's kept rows of Yp, accumulates w_j * row in fp32
 //             with j ascending, and writes y[t] once.  For k <= 8 the loads of
 //             all k rows of a column block are issued before the first
 //             multiply-add (one memory round trip per block instead of k).
-// Algorithmic bytes: dispatch T*d*s + R*d*s (+ T*k*4 index), combine
-// R*d*s + T*d*s (+ T*k*8 index/weights), s = element size.
+// Algorithmic bytes: dispatch U*d*s + R*d*s (+ T*k*4 index; U = tokens with a
+// kept row), combine R*d*s + T*d*s (+ T*k*8 index/weights), s = element size.
 #include "common.cuh"
 
 namespace moe {
@@ -44,6 +45,8 @@ dispatch_kernel(const uint4* __restrict__ x, int T, int nvec, int k,
                 my_row = -1;
             }
         }
+        // a token whose every slot was dropped is not read at all
+        if (!__any_sync(0xffffffffu, my_row >= 0)) continue;
         const uint4* src = x + (size_t)t * nvec;
         for (int c0 = 0; c0 < nvec; c0 += 32 * kU) {
             uint4 v[kU];
