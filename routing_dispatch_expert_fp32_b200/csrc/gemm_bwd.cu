@@ -16,7 +16,7 @@
 // offset), 8-row K groups 1 KB apart (stride byte offset).
 //
 // Same pipeline as the forward kernel (gemm_tc.cu): persistent CTAs, TMA
-// producer warp, one MMA-issuing thread, four epilogue warps draining two TMEM
+// producer warp, one MMA-issuing thread, eight epilogue warps draining two TMEM
 // accumulators, every wait bounded in time.  For the weight gradients a
 // group's last K block can run past the group's rows: its 16-row MMA steps
 // past the end are not issued, and in the step where the group ends the MMA
