@@ -69,6 +69,13 @@ constexpr int fixed_bytes() {
 
 enum Epi { EPI_BF16 = 0, EPI_BF16_RELU_MASK = 1, EPI_F32 = 2, EPI_BF16_ADD = 3 };
 
+// Input gradients of dense groups on the forward pass's 2-CTA pair tiles
+// (gemm_tc.cu; 0: the 1-CTA kernel below for every layout).
+#ifndef MOE_BWD_PAIR
+#define MOE_BWD_PAIR 1
+#endif
+constexpr bool kBwdPair = MOE_BWD_PAIR != 0;
+
 // Problem description of one launch.
 //   Fixed K: groups of rows from `offsets` (or one group of single_M rows
 //   when offsets is null), K = K_fix, B rows e*K_fix + k.
@@ -85,18 +92,6 @@ struct BwdArgs {
     const int32_t* offsets;
     int single_M, R_max, planes, plane_rows, slice_rows;
 };
-
-// MN-major operand descriptor, 128-byte swizzle: 64-element MN atoms 8 KB
-// apart, 8-row K groups 1 KB apart; +2 KB steps one K=16 slice.
-__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);      // start address
-    d |= static_cast<uint64_t>(MN_BOX_BYTES >> 4) << 16;       // leading byte offset
-    d |= static_cast<uint64_t>(1024 >> 4) << 32;               // stride byte offset
-    d |= static_cast<uint64_t>(1) << 46;                       // descriptor version
-    d |= static_cast<uint64_t>(2) << 61;                       // 128-byte swizzle
-    return d;
-}
 
 __device__ __forceinline__ float bf(uint32_t u, int hi) { return hi ? bf16hi(u) : bf16lo(u); }
 
@@ -510,20 +505,29 @@ int launch_ffn_backward_bf16(const void* Xp, const void* H, const void* dYp, con
     CUtensorMap a, b, c;
     std::memset(&c, 0, sizeof(c));  // unused by the bf16 epilogues
     const long long row_tiles = (long long)R_max / BM + E;
-    // dH: A = dYp [R_max, d] K-major; B = W2 as [E*d rows (K), F (N)]
-    if (make_tmap(&a, dYp, d, R_max, BM) != MOE_OK) return MOE_ERR_CUDA;
-    if (make_tmap(&b, W2, F, E * d, BK, MN_BOX) != MOE_OK) return MOE_ERR_CUDA;
-    int rc = launch_bwd<false, false, EPI_BF16_RELU_MASK>(
-        a, b, c, grouped(dH, H, 0, F, d, E, offsets, R_max), row_tiles * ((F + BN - 1) / BN),
-        st);
-    if (rc != MOE_OK) return rc;
-    // dXp: A = dH [R_max, F] K-major; B = W1 as [E*F rows (K), d (N)]
-    if (make_tmap(&a, dH, F, R_max, BM) != MOE_OK) return MOE_ERR_CUDA;
-    if (make_tmap(&b, W1, d, E * F, BK, MN_BOX) != MOE_OK) return MOE_ERR_CUDA;
-    rc = launch_bwd<false, false, EPI_BF16>(a, b, c, grouped(dXp, nullptr, 0, d, F, E, offsets,
-                                                             R_max),
-                                           row_tiles * ((d + BN - 1) / BN), st);
-    if (rc != MOE_OK) return rc;
+    int rc;
+    if (kBwdPair && offsets != nullptr && gemm_groups_dense(R_max, E)) {
+        // dense groups: the forward pass's 2-CTA 256 x 256 tiles, weights read N-major
+        rc = launch_gemm_pair_nmajor_bf16(dYp, W2, dH, F, d, E, offsets, R_max, H, st);
+        if (rc != MOE_OK) return rc;
+        rc = launch_gemm_pair_nmajor_bf16(dH, W1, dXp, d, F, E, offsets, R_max, nullptr, st);
+        if (rc != MOE_OK) return rc;
+    } else {
+        // dH: A = dYp [R_max, d] K-major; B = W2 as [E*d rows (K), F (N)]
+        if (make_tmap(&a, dYp, d, R_max, BM) != MOE_OK) return MOE_ERR_CUDA;
+        if (make_tmap(&b, W2, F, E * d, BK, MN_BOX) != MOE_OK) return MOE_ERR_CUDA;
+        rc = launch_bwd<false, false, EPI_BF16_RELU_MASK>(
+            a, b, c, grouped(dH, H, 0, F, d, E, offsets, R_max), row_tiles * ((F + BN - 1) / BN),
+            st);
+        if (rc != MOE_OK) return rc;
+        // dXp: A = dH [R_max, F] K-major; B = W1 as [E*F rows (K), d (N)]
+        if (make_tmap(&a, dH, F, R_max, BM) != MOE_OK) return MOE_ERR_CUDA;
+        if (make_tmap(&b, W1, d, E * F, BK, MN_BOX) != MOE_OK) return MOE_ERR_CUDA;
+        rc = launch_bwd<false, false, EPI_BF16>(a, b, c, grouped(dXp, nullptr, 0, d, F, E,
+                                                                 offsets, R_max),
+                                               row_tiles * ((d + BN - 1) / BN), st);
+        if (rc != MOE_OK) return rc;
+    }
     if (dW2) {  // A = dYp rows as [K, M=d], B = H rows as [K, N=F]
         if (make_tmap(&a, dYp, d, R_max, BK, MN_BOX) != MOE_OK) return MOE_ERR_CUDA;
         if (make_tmap(&b, H, F, R_max, BK, MN_BOX) != MOE_OK) return MOE_ERR_CUDA;

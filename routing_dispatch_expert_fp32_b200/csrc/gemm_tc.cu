@@ -323,6 +323,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
 // which reads both CTAs' shared memory and writes each CTA's 128 rows into that
 // CTA's TMEM.  Each CTA streams half the B bytes of a 1-CTA 128x256 tile for
 // the same MMA work, so a 6-deep ring fits and hides more latency.
+//
+// The same kernel serves the input gradients of the expert backward
+// (B_MN: B read N-major, as the forward weights lie: [E*K rows][N], each CTA's
+// 128 columns as two 64 x 64 boxes; MASK: the result zeroed where the forward
+// activation Hmask was not positive, for dH = (dYp . W2_e) * [H > 0]).
 namespace pair {
 
 constexpr int kStages = 6;
@@ -395,11 +400,12 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
                  : "memory");
 }
 
-template <bool RELU>
+template <bool RELU, bool B_MN = false, bool MASK = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b, __nv_bfloat16* __restrict__ C, int N,
-                int K, int E, const int32_t* __restrict__ offsets, int R_max, int part, int32_t* err) {
+                int K, int E, const int32_t* __restrict__ offsets, int R_max, int part,
+                const __nv_bfloat16* __restrict__ Hmask, int32_t* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~static_cast<uintptr_t>(1023u));
@@ -466,7 +472,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
             for (int tile = first; ok && tile < total; tile += npairs) {
                 const TileCoord c = tile_coord(tile, s_prefix, E, offsets, 0, BM, bn, nt, part);
                 const int a_row = c.row0 + HALF * (int)rank;
-                const int b_row = c.e * N + c.n0 + b_half * (int)rank;
+                const int b_row = c.e * N + c.n0 + b_half * (int)rank;  // K-major B
+                const int b_col = c.n0 + b_half * (int)rank;            // N-major B
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, err)) {
                         ok = false;
@@ -475,7 +482,15 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const uint32_t lbar = map_to(smem_u32(full + stage), 0);
                     if (leader) mbar_arrive_expect_tx(full + stage, pair_tx);
                     tma_load_2d_pair(sA + stage * A_BYTES, &tmap_a, lbar, kb * BK, a_row);
-                    tma_load_2d_pair(sB + stage * B_BYTES, mb, lbar, kb * BK, b_row);
+                    if constexpr (B_MN) {
+                        // K rows c.e*K + kb*BK.. of the weight, this CTA's 128 columns
+                        const int k_row = c.e * K + kb * BK;
+                        tma_load_2d_pair(sB + stage * B_BYTES, mb, lbar, b_col, k_row);
+                        tma_load_2d_pair(sB + stage * B_BYTES + kMnAtomBytes, mb, lbar,
+                                         b_col + 64, k_row);
+                    } else {
+                        tma_load_2d_pair(sB + stage * B_BYTES, mb, lbar, kb * BK, b_row);
+                    }
                     ++issued;
                     if (++stage == kStages) {
                         stage = 0;
@@ -501,7 +516,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issuer (leader only)
-            const uint32_t idesc = idesc_bf16(BM, bn);
+            const uint32_t idesc = idesc_bf16(BM, bn) | (B_MN ? (1u << 16) : 0u);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -521,8 +536,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        mma_pair(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc,
-                                 (kb | kk) != 0 ? 1u : 0u);
+                        mma_pair(d_tmem, sw128_desc(a0 + kk * 32),
+                                 B_MN ? sw128_mn_desc(b0 + kk * 2048) : sw128_desc(b0 + kk * 32),
+                                 idesc, (kb | kk) != 0 ? 1u : 0u);
                     commit_both(empty + stage);
                     if (++stage == kStages) {
                         stage = 0;
@@ -548,11 +564,45 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a,
             const int r_tile = HALF * (int)rank + row;  // row inside the 256-row tile
             const bool row_ok = r_tile < c.rows;
             __nv_bfloat16* crow = C + static_cast<size_t>(c.row0 + (row_ok ? r_tile : 0)) * N;
+            // MASK: bit i of hm[w] says column c.n0 + 32 w + i of this row has H > 0
+            uint32_t hm[BN / 32];
+#pragma unroll
+            for (int w = 0; w < BN / 32; ++w) hm[w] = 0u;
+            if constexpr (MASK) {
+                if (row_ok) {
+                    const uint4* h = reinterpret_cast<const uint4*>(
+                        Hmask + static_cast<size_t>(c.row0 + r_tile) * N + c.n0);
+                    const int nv = min(BN, N - c.n0) / 8;
+#pragma unroll
+                    for (int w = 0; w < BN / 32; ++w) {
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq) {
+                            const int q = 4 * w + qq;
+                            const uint4 v = q < nv ? ldg_nc_v4(h + q) : make_uint4(0, 0, 0, 0);
+                            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+                            uint32_t bits = 0;
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                bits |= ((i & 1 ? bf16hi(u[i >> 1]) : bf16lo(u[i >> 1])) > 0.0f
+                                             ? 1u : 0u) << i;
+                            hm[w] |= bits << (qq * 8);
+                        }
+                    }
+                }
+            }
 #pragma unroll 1
             for (int cc = 0; cc < bn; cc += 32) {
                 uint32_t r[32];
                 tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(acc * BN + cc), r);
                 const int col = c.n0 + cc;
+                if constexpr (MASK) {
+                    const uint32_t mw = hm[0];  // this 32-column block's bits
+#pragma unroll
+                    for (int w = 0; w + 1 < BN / 32; ++w) hm[w] = hm[w + 1];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (!((mw >> i) & 1u)) r[i] = 0u;
+                }
                 if (row_ok && col < N) Store32<__nv_bfloat16, RELU>::run(crow + col, r, N - col);
             }
             tc_fence_before();
@@ -615,7 +665,30 @@ static int launch_pair(const void* A, const void* B, __nv_bfloat16* C, int N, in
     int pairs = (int)(ub < pairs_max ? ub : pairs_max);
     pairs = test_cap(2 * pairs) / 2 > 0 ? test_cap(2 * pairs) / 2 : 1;
     return launch_pdl(kern, 2 * pairs, kThreads, smem, st, ta, tb, C, N, K, E, offsets, R_max,
-                      part, device_error_word());
+                      part, static_cast<const __nv_bfloat16*>(nullptr), device_error_word());
+}
+
+// Pair tiles with the weights read N-major: C[rows of group e] = A . B_e with
+// B_e rows [e*K, e*K + K) of a [E*K, N] matrix, optionally masked by Hmask > 0.
+template <bool MASK>
+static int launch_pair_nmajor(const void* A, const void* B, __nv_bfloat16* C, int N, int K,
+                              int E, const int32_t* offsets, int R_max, const void* Hmask,
+                              cudaStream_t st) {
+    if (R_max <= 0 || N <= 0) return MOE_OK;
+    CUtensorMap ta, tb;
+    if (make_tmap(&ta, A, K, R_max, pair::HALF) != MOE_OK) return MOE_ERR_CUDA;
+    if (make_tmap(&tb, B, N, E * K, BK, 64) != MOE_OK) return MOE_ERR_CUDA;
+    const int smem = pair::smem_bytes(E);
+    auto kern = pair::gemm_tc2_kernel<false, true, MASK>;
+    if (ensure_smem<pair::gemm_tc2_kernel<false, true, MASK>>(smem) != MOE_OK) return MOE_ERR_CUDA;
+    const int nt = (N + pair::BN - 1) / pair::BN;
+    const long long ub = ((long long)R_max / pair::BM + E) * nt;
+    const int pairs_max = num_sms() / 2;
+    int pairs = (int)(ub < pairs_max ? ub : pairs_max);
+    pairs = test_cap(2 * pairs) / 2 > 0 ? test_cap(2 * pairs) / 2 : 1;
+    return launch_pdl(kern, 2 * pairs, kThreads, smem, st, ta, tb, C, N, K, E, offsets, R_max,
+                      (int)PART_ALL, static_cast<const __nv_bfloat16*>(Hmask),
+                      device_error_word());
 }
 
 }  // namespace tc
@@ -623,6 +696,19 @@ static int launch_pair(const void* A, const void* B, __nv_bfloat16* C, int N, in
 #ifdef MOE_TEST_HOOKS
 int test_stall_tc(int v) { return tc::set_test_stall(v); }
 #endif
+
+bool gemm_groups_dense(int R_max, int E) {
+    return (long long)R_max >= tc::kPairMinRowsPerGroup * (long long)E;
+}
+
+int launch_gemm_pair_nmajor_bf16(const void* A, const void* B, void* C, int N, int K, int E,
+                                 const int32_t* offsets, int R_max, const void* Hmask,
+                                 cudaStream_t st) {
+    __nv_bfloat16* Cb = static_cast<__nv_bfloat16*>(C);
+    if (Hmask)
+        return tc::launch_pair_nmajor<true>(A, B, Cb, N, K, E, offsets, R_max, Hmask, st);
+    return tc::launch_pair_nmajor<false>(A, B, Cb, N, K, E, offsets, R_max, nullptr, st);
+}
 
 int launch_gemm_tc_bf16(const void* A, const void* B, void* C, bool out_f32, int N, int K, int E,
                         const int32_t* offsets, int single_M, int R_max, bool relu,

@@ -149,7 +149,21 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     d |= static_cast<uint64_t>(2) << 61;                  // 128-byte swizzle
     return d;
 }
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both K-major.
+// MN-major operand descriptor, 128-byte swizzle: 64-element MN atoms (one
+// 64 x 64 TMA box each) 8 KB apart, 8-row K groups 1 KB apart; +2 KB steps one
+// K=16 slice.
+constexpr int kMnAtomBytes = 64 * BK * 2;  // 8 KB
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);      // start address
+    d |= static_cast<uint64_t>(kMnAtomBytes >> 4) << 16;       // leading byte offset
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;               // stride byte offset
+    d |= static_cast<uint64_t>(1) << 46;                       // descriptor version
+    d |= static_cast<uint64_t>(2) << 61;                       // 128-byte swizzle
+    return d;
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major (bit 15 / bit 16 mark an MN-major A / B).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);

@@ -62,17 +62,23 @@ def run_ffn_bwd(moe, Xp, H, dYp, W1, W2, offsets, Rmax, dtype, weight_grads=True
     return out
 
 
-@pytest.mark.parametrize("sizes,d,F,dtype", [
-    ([0, 1, 127, 128, 129, 300], 200, 328, "bf16"),
-    ([5, 0, 260], 64, 256, "bf16"),
-    ([513], 1024, 512, "bf16"),
-    ([3, 77, 131, 0, 0, 256, 1], 136, 520, "bf16"),
-    ([0, 0, 0], 64, 64, "bf16"),
-    ([64, 65, 63], 8, 16, "bf16"),
-    ([40, 90, 1], 64, 128, "f32"),
-    ([0, 65, 200], 72, 100, "f32"),
+@pytest.mark.parametrize("sizes,d,F,dtype,rmax", [
+    ([0, 1, 127, 128, 129, 300], 200, 328, "bf16", 0),
+    ([5, 0, 260], 64, 256, "bf16", 0),
+    ([513], 1024, 512, "bf16", 0),
+    ([3, 77, 131, 0, 0, 256, 1], 136, 520, "bf16", 0),
+    ([0, 0, 0], 64, 64, "bf16", 0),
+    ([64, 65, 63], 8, 16, "bf16", 0),
+    ([40, 90, 1], 64, 128, "f32", 0),
+    ([0, 65, 200], 72, 100, "f32", 0),
+    # row capacity >= 1024 per group: the input gradients take the 2-CTA pair
+    # tiles (weights read N-major), with ragged groups, an empty one, N and K
+    # not multiples of the tile
+    ([1000, 1300], 200, 328, "bf16", 2048),
+    ([0, 700, 1900, 3], 136, 520, "bf16", 4096),
+    ([2048], 64, 256, "bf16", 2048),
 ])
-def test_ffn_backward_small_shapes_elementwise(moe, sizes, d, F, dtype):
+def test_ffn_backward_small_shapes_elementwise(moe, sizes, d, F, dtype, rmax):
     E, R = len(sizes), sum(sizes)
     offsets = np.array([0] + np.cumsum(sizes).tolist(), np.int32)
     Xp = rand((R, d), 1.0, dtype, 11)
@@ -80,7 +86,7 @@ def test_ffn_backward_small_shapes_elementwise(moe, sizes, d, F, dtype):
     dYp = rand((R, d), 1.0, dtype, 13)
     W1 = rand((E, F, d), d ** -0.5, dtype, 14)
     W2 = rand((E, d, F), F ** -0.5, dtype, 15)
-    Rmax = R + 37
+    Rmax = max(R + 37, rmax)
     g = run_ffn_bwd(moe, Xp, H, dYp, W1, W2, offsets, Rmax, dtype)
     tol = dict(max_abs_frac=1e-4, mean_rel=1e-5) if dtype == "f32" else {}
     if R:
