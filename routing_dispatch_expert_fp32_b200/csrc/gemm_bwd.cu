@@ -506,28 +506,30 @@ int launch_ffn_backward_bf16(const void* Xp, const void* H, const void* dYp, con
     std::memset(&c, 0, sizeof(c));  // unused by the bf16 epilogues
     const long long row_tiles = (long long)R_max / BM + E;
     int rc;
-    if (kBwdPair && offsets != nullptr && gemm_groups_dense(R_max, E)) {
-        // dense groups: the forward pass's 2-CTA 256 x 256 tiles, weights read N-major
+    // Each input gradient takes the forward pass's 2-CTA 256 x 256 tiles (weights
+    // read N-major) where the forward pass would for its N, else 1-CTA tiles.
+    // dH: A = dYp [R_max, d] K-major; B = W2 as [E*d rows (K), F (N)]
+    if (kBwdPair && offsets != nullptr && gemm_pair_tiles(R_max, E, F)) {
         rc = launch_gemm_pair_nmajor_bf16(dYp, W2, dH, F, d, E, offsets, R_max, H, st);
-        if (rc != MOE_OK) return rc;
-        rc = launch_gemm_pair_nmajor_bf16(dH, W1, dXp, d, F, E, offsets, R_max, nullptr, st);
-        if (rc != MOE_OK) return rc;
     } else {
-        // dH: A = dYp [R_max, d] K-major; B = W2 as [E*d rows (K), F (N)]
         if (make_tmap(&a, dYp, d, R_max, BM) != MOE_OK) return MOE_ERR_CUDA;
         if (make_tmap(&b, W2, F, E * d, BK, MN_BOX) != MOE_OK) return MOE_ERR_CUDA;
         rc = launch_bwd<false, false, EPI_BF16_RELU_MASK>(
             a, b, c, grouped(dH, H, 0, F, d, E, offsets, R_max), row_tiles * ((F + BN - 1) / BN),
             st);
-        if (rc != MOE_OK) return rc;
-        // dXp: A = dH [R_max, F] K-major; B = W1 as [E*F rows (K), d (N)]
+    }
+    if (rc != MOE_OK) return rc;
+    // dXp: A = dH [R_max, F] K-major; B = W1 as [E*F rows (K), d (N)]
+    if (kBwdPair && offsets != nullptr && gemm_pair_tiles(R_max, E, d)) {
+        rc = launch_gemm_pair_nmajor_bf16(dH, W1, dXp, d, F, E, offsets, R_max, nullptr, st);
+    } else {
         if (make_tmap(&a, dH, F, R_max, BM) != MOE_OK) return MOE_ERR_CUDA;
         if (make_tmap(&b, W1, d, E * F, BK, MN_BOX) != MOE_OK) return MOE_ERR_CUDA;
         rc = launch_bwd<false, false, EPI_BF16>(a, b, c, grouped(dXp, nullptr, 0, d, F, E,
                                                                  offsets, R_max),
                                                row_tiles * ((d + BN - 1) / BN), st);
-        if (rc != MOE_OK) return rc;
     }
+    if (rc != MOE_OK) return rc;
     if (dW2) {  // A = dYp rows as [K, M=d], B = H rows as [K, N=F]
         if (make_tmap(&a, dYp, d, R_max, BK, MN_BOX) != MOE_OK) return MOE_ERR_CUDA;
         if (make_tmap(&b, H, F, R_max, BK, MN_BOX) != MOE_OK) return MOE_ERR_CUDA;

@@ -697,8 +697,10 @@ static int launch_pair_nmajor(const void* A, const void* B, __nv_bfloat16* C, in
 int test_stall_tc(int v) { return tc::set_test_stall(v); }
 #endif
 
-bool gemm_groups_dense(int R_max, int E) {
-    return (long long)R_max >= tc::kPairMinRowsPerGroup * (long long)E;
+bool gemm_pair_tiles(int R_max, int E, int N) {
+    const long long tiles_1cta = ((long long)R_max / tc::BM + E) * ((N + 255) / 256);
+    return (long long)R_max >= tc::kPairMinRowsPerGroup * (long long)E ||
+           tiles_1cta < 3LL * num_sms();
 }
 
 int launch_gemm_pair_nmajor_bf16(const void* A, const void* B, void* C, int N, int K, int E,

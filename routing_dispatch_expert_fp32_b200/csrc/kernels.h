@@ -25,11 +25,12 @@ int launch_gemm_tc_bf16(const void* A, const void* B, void* C, bool out_f32, int
                         const int32_t* offsets, int single_M, int R_max, bool relu,
                         cudaStream_t st);
 
-// Groups dense enough for the 2-CTA pair tiles (rows per group on average), and
-// the pair GEMM with the weights read N-major ([E*K, N], rows e*K.. for group
-// e), C bf16, zeroed where Hmask (when non-null, [R, N] bf16) is not positive
-// (gemm_tc.cu; the expert backward's input gradients).
-bool gemm_groups_dense(int R_max, int E);
+// Whether a grouped GEMM of N columns takes the 2-CTA pair tiles (the forward
+// pass's rule: groups dense on average, or 128-row tiles filling fewer than
+// three waves), and the pair GEMM with the weights read N-major ([E*K, N], rows
+// e*K.. for group e), C bf16, zeroed where Hmask (when non-null, [R, N] bf16)
+// is not positive (gemm_tc.cu; the expert backward's input gradients).
+bool gemm_pair_tiles(int R_max, int E, int N);
 int launch_gemm_pair_nmajor_bf16(const void* A, const void* B, void* C, int N, int K, int E,
                                  const int32_t* offsets, int R_max, const void* Hmask,
                                  cudaStream_t st);

@@ -77,6 +77,9 @@ def run_ffn_bwd(moe, Xp, H, dYp, W1, W2, offsets, Rmax, dtype, weight_grads=True
     ([1000, 1300], 200, 328, "bf16", 2048),
     ([0, 700, 1900, 3], 136, 520, "bf16", 4096),
     ([2048], 64, 256, "bf16", 2048),
+    # 460 groups of 0-4 rows: more than three waves of 128-row tiles, so both
+    # input gradients take the 1-CTA kernel
+    ([int(v) for v in np.random.default_rng(7).integers(0, 5, 460)], 256, 256, "bf16", 0),
 ])
 def test_ffn_backward_small_shapes_elementwise(moe, sizes, d, F, dtype, rmax):
     E, R = len(sizes), sum(sizes)
