@@ -32,9 +32,11 @@ popularity_kernel(const int32_t* __restrict__ counts, int E, int32_t* __restrict
         const int32_t c = counts[e];
         hist[(size_t)slot * E + e] = c;
         long long sum = c;
+        // rows of the n - 1 earlier live steps: slot - 1, slot - 2, ... wrapped
+        // into [0, W) (no 64-bit division per row)
 #pragma unroll 4
-        for (long long i = 1; i < n; ++i) {
-            const int s = (int)((step - i) % W);
+        for (int i = 1; i < (int)n; ++i) {
+            const int s = slot - i < 0 ? slot - i + W : slot - i;
             sum += hist[(size_t)s * E + e];
         }
         s_sum[e] = sum;
